@@ -1,0 +1,311 @@
+"""Pins for the CPU oracle (no GPU).
+
+Each test checks the oracle against something other than itself: a library
+special case (torch's float8_e4m3fn cast, scipy's Hadamard matrix and
+logsumexp, torch's float64 scaled_dot_product_attention), a closed form, an
+invariant of softmax attention, or brute force on tiny inputs.
+"""
+import os
+
+import numpy as np
+import pytest
+import scipy.linalg
+import scipy.special
+import torch
+
+import oracle
+import workloads
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _t2e4m3_codes(x32: np.ndarray) -> np.ndarray:
+    return torch.from_numpy(np.ascontiguousarray(x32, dtype=np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+# ------------------------------------------------------------------ codec
+def test_e4m3_decode_all_256_match_torch():
+    codes = np.arange(256, dtype=np.uint8)
+    mine = oracle.e4m3_decode(codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(np.isnan(mine), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(mine[ok], ref[ok])
+    assert np.isnan(mine[0x7F]) and np.isnan(mine[0xFF])
+    assert mine[0x7E] == 448.0 and mine[1] == 2.0 ** -9
+
+
+def test_e4m3_encode_random_and_ties_match_torch():
+    rng = np.random.default_rng(0)
+    mag = np.exp2(rng.uniform(-13, 8.85, 200_000))  # below subnormals .. 460
+    x = (mag * rng.choice([-1.0, 1.0], mag.size)).astype(np.float32)
+    # every midpoint between consecutive finite codes (ties) and the codes
+    vals = oracle.e4m3_decode(np.arange(0, 127, dtype=np.uint8))
+    mids = ((vals[:-1] + vals[1:]) / 2).astype(np.float32)
+    x = np.concatenate([x, mids, -mids, vals.astype(np.float32), np.float32([0.0, -0.0])])
+    assert np.all(np.abs(x) < 464)  # torch turns >= 464 into NaN; we saturate
+    mine = oracle.e4m3_encode(x.astype(np.float64))
+    assert np.array_equal(mine, _t2e4m3_codes(x))
+
+
+def test_e4m3_encode_saturates_and_nan():
+    assert oracle.e4m3_encode(np.array([464.0, 1e30, np.inf]))[0] == 0x7E
+    assert list(oracle.e4m3_encode(np.array([-500.0, np.inf, np.nan]))) == [0xFE, 0x7E, 0x7F]
+
+
+def test_golden_powers_of_two_grow_by_8_per_doubling():
+    rows = [l.split() for l in open(os.path.join(GOLDEN, "e4m3_powers_of_two.txt")) if l.strip() and not l.startswith("#")]
+    for k, val, code in rows:
+        assert float(val) == 2.0 ** int(k)
+        assert oracle.e4m3_encode(np.array([float(val)]))[0] == int(code)
+        assert oracle.e4m3_decode(np.array([int(code)], dtype=np.uint8))[0] == float(val)
+    # the doubling rule for arbitrary normal values in [2^-6, 224]
+    rng = np.random.default_rng(1)
+    x = np.exp2(rng.uniform(-6, 7.8, 5000))
+    c1 = oracle.e4m3_encode(x).astype(int)
+    c2 = oracle.e4m3_encode(2 * x).astype(int)
+    assert np.all(c2 == c1 + 8)
+
+
+# ---------------------------------------------------------------- Hadamard
+def test_fwht_matches_scipy_hadamard():
+    rng = np.random.default_rng(2)
+    x = rng.standard_normal((7, 128)).astype(np.float32)
+    H = scipy.linalg.hadamard(128).astype(np.float64)
+    mine = oracle.fwht128(x).astype(np.float64)
+    ref = x.astype(np.float64) @ H.T
+    assert np.allclose(mine, ref, rtol=0, atol=1e-4)
+    twice = oracle.fwht128(oracle.fwht128(x)).astype(np.float64)
+    assert np.allclose(twice, 128.0 * x, rtol=0, atol=1e-3)
+
+
+def test_hadamard_preserves_scores_up_to_128():
+    rng = np.random.default_rng(3)
+    q = rng.standard_normal((5, 128))
+    k = rng.standard_normal((6, 128))
+    H = scipy.linalg.hadamard(128).astype(np.float64)
+    assert np.allclose((q @ H.T) @ (k @ H.T).T, 128.0 * q @ k.T, atol=1e-9)
+
+
+# --------------------------------------------------------------- quantiser
+@pytest.mark.parametrize("hadamard", [False, True])
+@pytest.mark.parametrize("src", ["f32", "bf16"])
+def test_quantize_matches_torch_cast(hadamard, src):
+    q, _, _ = workloads.make_custom(1, 300, 300, 3, 3, 128, 128, seed=5)
+    x32 = q.numpy().astype(np.float32)
+    if src == "bf16":
+        xb = torch.from_numpy(x32).to(torch.bfloat16)
+        xin = xb.view(torch.int16).numpy().view(np.uint16)
+        x32 = xb.to(torch.float32).numpy()
+    else:
+        xin = x32
+    codes, ds = oracle.quantize_fp8(xin, hadamard=hadamard)
+    if hadamard:
+        H = scipy.linalg.hadamard(128).astype(np.float64)
+        rot = oracle.fwht128(x32)
+        assert np.allclose(rot.astype(np.float64), x32.astype(np.float64) @ H.T, atol=1e-4)
+        x32 = rot
+    amax = np.float32(np.abs(x32).max())
+    inv = np.float32(np.float32(448.0) / amax)
+    scaled = (x32 * inv).astype(np.float32)
+    assert np.array_equal(codes, _t2e4m3_codes(scaled))
+    exp_ds = np.float32(amax / np.float32(448.0))
+    if hadamard:
+        exp_ds = np.float32(exp_ds * np.float32(2.0 ** -3.5))
+    assert ds == exp_ds
+    # the largest magnitude maps to the largest finite code
+    assert (codes & 0x7F).max() == 0x7E
+    # dequantised values are within half an e4m3 step (relative 1/16)
+    deq = oracle.dequant_e4m3(codes, float(amax / np.float32(448.0)))
+    big = np.abs(x32) > amax * 2.0 ** -6
+    assert np.all(np.abs(deq[big] - x32[big]) <= np.abs(x32[big]) / 16 * 1.0001 + 1e-12)
+
+
+def test_quantize_zero_tensor():
+    codes, ds = oracle.quantize_fp8(np.zeros((4, 128), dtype=np.float32))
+    assert not codes.any() and ds == 0.0
+
+
+# ---------------------------------------------------------------- R1 exact
+@pytest.mark.parametrize("shape", [(1, 37, 37, 2, 2, 16, 16), (2, 20, 33, 4, 2, 24, 8), (1, 33, 20, 3, 1, 8, 12)])
+def test_attn_ref_matches_numpy_brute_force(shape):
+    B, Sq, Sk, Hq, Hkv, dqk, dv = shape
+    q, k, v = (t.numpy() for t in workloads.make_custom(B, Sq, Sk, Hq, Hkv, dqk, dv, seed=7))
+    for causal in (True, False):
+        o, l = oracle.attn_ref(q, k, v, causal=causal)
+        ob, lb = oracle.brute_attn(q, k, v, causal=causal)
+        assert np.allclose(o, ob, atol=1e-12)
+        assert np.array_equal(np.isinf(l), np.isinf(lb))
+        fin = np.isfinite(lb)
+        assert np.allclose(l[fin], lb[fin], atol=1e-12)
+
+
+def test_attn_ref_matches_torch_sdpa_float64():
+    q, k, v = workloads.make_custom(2, 50, 50, 4, 4, 32, 32, seed=8)
+    o, l = oracle.attn_ref(q.numpy(), k.numpy(), v.numpy(), causal=True)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        q.double().transpose(1, 2), k.double().transpose(1, 2), v.double().transpose(1, 2), is_causal=True
+    ).transpose(1, 2)
+    assert np.allclose(o, ref.numpy(), atol=1e-12)
+
+
+def test_attn_ref_lse_is_logsumexp_of_scores():
+    q, k, v = (t.numpy().astype(np.float64) for t in workloads.make_custom(1, 40, 40, 1, 1, 16, 16, seed=9))
+    o, l = oracle.attn_ref(q, k, v, causal=True)
+    s = (q[0, :, 0] @ k[0, :, 0].T) / 4.0
+    for i in range(40):
+        assert abs(l[0, 0, i] - scipy.special.logsumexp(s[i, : i + 1])) < 1e-12
+
+
+def test_attn_ref_invariants():
+    B, S, H, d = 1, 64, 2, 16
+    q, k, v = (t.numpy().astype(np.float64) for t in workloads.make_custom(B, S, S, H, H, d, d, seed=10))
+    # (1) probabilities of each row sum to 1: V = ones gives o = 1
+    o, _ = oracle.attn_ref(q, k, np.ones_like(v))
+    assert np.allclose(o, 1.0, atol=1e-14)
+    # (2) causal query row 0 returns v_0
+    o, l = oracle.attn_ref(q, k, v)
+    assert np.allclose(o[:, 0], v[:, 0], atol=1e-14)
+    # (3) constant K: uniform weights, o_i = mean(v_0..v_i), lse = s + ln(i+1)
+    kc = np.broadcast_to(k[:, :1], k.shape).copy()
+    o, l = oracle.attn_ref(q, kc, v)
+    run = np.cumsum(v, axis=1) / np.arange(1, S + 1)[None, :, None, None]
+    assert np.allclose(o, run, atol=1e-13)
+    s0 = np.einsum("bihd,bhd->bhi", q, kc[:, 0]) / np.sqrt(d)
+    assert np.allclose(l, s0 + np.log(np.arange(1, S + 1))[None, None, :], atol=1e-12)
+
+
+def test_attn_ref_gqa_equals_repeated_heads():
+    q, k, v = (t.numpy() for t in workloads.make_custom(1, 30, 30, 4, 1, 16, 16, seed=11))
+    o1, l1 = oracle.attn_ref(q, k, v)
+    o2, l2 = oracle.attn_ref(q, np.repeat(k, 4, axis=2), np.repeat(v, 4, axis=2))
+    assert np.allclose(o1, o2, atol=1e-15) and np.allclose(l1, l2, atol=1e-15)
+
+
+def test_attn_ref_empty_rows_when_sq_exceeds_sk():
+    q, k, v = (t.numpy() for t in workloads.make_custom(1, 10, 4, 1, 1, 8, 8, seed=12))
+    o, l = oracle.attn_ref(q, k, v, causal=True)
+    assert np.all(o[0, :6] == 0) and np.all(np.isneginf(l[0, 0, :6]))
+    assert np.allclose(o[0, 6], v[0, 0])
+
+
+def test_attn_ref_row_sampling_matches_full():
+    q, k, v = (t.numpy() for t in workloads.make_custom(2, 70, 70, 2, 1, 16, 8, seed=13))
+    o, l = oracle.attn_ref(q, k, v)
+    rows = workloads.sample_rows(2, 2, 70, every=16).numpy()
+    os_, ls = oracle.attn_ref(q, k, v, rows=rows)
+    b, rem = rows // (2 * 70), rows % (2 * 70)
+    h, i = rem // 70, rem % 70
+    assert np.allclose(os_, o[b, i, h], atol=0) and np.allclose(ls, l[b, h, i], atol=0)
+
+
+# ------------------------------------------------------------ R2 FP8 path
+@pytest.mark.parametrize("block_scale", [True, False])
+@pytest.mark.parametrize("T", [0, 8])
+def test_emul_without_rounding_equals_exact(block_scale, T):
+    q, k, v = (t.numpy() for t in workloads.make_custom(1, 300, 300, 2, 1, 32, 16, seed=14, std=1.5))
+    o, l = oracle.attn_ref(q, k, v)
+    oe, le = oracle.attn_fp8_emul(q, k, v, mode=oracle.MODE_NOROUND, block_scale=block_scale, T=T)
+    assert np.allclose(oe, o, atol=1e-12) and np.allclose(le, l, atol=1e-12)
+
+
+@pytest.mark.parametrize("mode", [oracle.MODE_EXACT, oracle.MODE_LEANP])
+@pytest.mark.parametrize("block_scale", [True, False])
+def test_emul_divides_by_rounded_sum(mode, block_scale):
+    # V = ones: o = sum(w p~) / sum(w p~) = 1 exactly only when the division
+    # uses the sum of the *rounded* probabilities (an unrounded sum is off by
+    # the FP8 rounding error, ~1e-2).
+    q, k, v = (t.numpy() for t in workloads.make_custom(1, 200, 200, 2, 2, 32, 8, seed=15))
+    oe, _ = oracle.attn_fp8_emul(q, k, np.ones_like(v), mode=mode, block_scale=block_scale)
+    assert np.allclose(oe, 1.0, atol=1e-14)
+
+
+def _row_scores(q, k, i, scale):
+    return (q[0, i, 0].astype(np.float64) @ k[0, : i + 1, 0].astype(np.float64).T) * scale * np.log2(np.e)
+
+
+def test_leanp_closed_form_and_mitchell_bounds():
+    S, d = 256, 32
+    q, k, v = (t.numpy() for t in workloads.make_custom(1, S, S, 1, 1, d, 8, seed=16, std=1.3))
+    scale = 1 / np.sqrt(d)
+    i = S - 1
+    _, _, p = oracle.attn_fp8_emul(q, k, v, mode=oracle.MODE_LEANP, rows=[i], want_p=True)
+    y = _row_scores(q, k, i, scale)
+    T = 8
+    for j0 in range(0, S, 64):
+        yb = y[j0 : j0 + 64]
+        e = np.ceil(yb.max()) - T
+        z = yb - e
+        pb = p[j0 : j0 + 64]
+        # block maximum lands in (2^(T-1), 2^T]
+        assert 2.0 ** (T - 1) < pb[np.argmax(yb)] * 1.0000001 and pb.max() <= 2.0 ** T
+        normal = z > -6
+        # piecewise-linear 2^f ~ 1+f between integers, +-1/16 code from rounding
+        ratio = pb[normal] / np.exp2(z[normal])
+        assert np.all(ratio >= 2.0 ** (-1 / 16) * 0.999999)
+        assert np.all(ratio <= 1.0615 * 2.0 ** (1 / 16))
+    # at integer log2 values the code is 8t+56 and the value is exactly 2^t
+    codes = oracle.e4m3_encode(np.exp2(np.arange(-6, 9, dtype=np.float64)))
+    assert list(codes) == [8 * t + 56 for t in range(-6, 9)]
+
+
+def test_exact_mode_p_is_rounded_exp2():
+    S, d = 192, 32
+    q, k, v = (t.numpy() for t in workloads.make_custom(1, S, S, 1, 1, d, 8, seed=17))
+    i = S - 1
+    _, _, p = oracle.attn_fp8_emul(q, k, v, mode=oracle.MODE_EXACT, T=8, rows=[i], want_p=True)
+    y = _row_scores(q, k, i, 1 / np.sqrt(d))
+    for j0 in range(0, S, 64):
+        z = y[j0 : j0 + 64] - (np.ceil(y[j0 : j0 + 64].max()) - 8)
+        # torch cast of fp32(2^z) is the library special case (z never hits
+        # an fp32 rounding of a tie here)
+        ref = torch.from_numpy(np.exp2(z).astype(np.float32)).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+        assert np.array_equal(p[j0 : j0 + 64], ref)
+
+
+def test_emul_block_order_independent():
+    # Non-causal: R2 depends on the set of 64-key blocks, not their order.
+    S = 256
+    q, k, v = (t.numpy() for t in workloads.make_custom(1, 16, S, 1, 1, 32, 8, seed=18, std=1.4))
+    perm = np.concatenate([np.arange(b * 64, b * 64 + 64) for b in (2, 0, 3, 1)])
+    for mode in (oracle.MODE_EXACT, oracle.MODE_LEANP):
+        o1, l1 = oracle.attn_fp8_emul(q, k, v, causal=False, mode=mode)
+        o2, l2 = oracle.attn_fp8_emul(q, k[:, perm], v[:, perm], causal=False, mode=mode)
+        assert np.allclose(o1, o2, atol=1e-13) and np.allclose(l1, l2, atol=1e-13)
+
+
+def test_emul_headroom_invariance_without_clamping():
+    # Narrow score range: no code reaches the clamp at 0, so moving the
+    # headroom T by whole steps only shifts codes by multiples of 8.
+    q, k, v = (t.numpy() for t in workloads.make_custom(1, 128, 128, 1, 1, 32, 8, seed=19, std=0.3))
+    for mode in (oracle.MODE_EXACT, oracle.MODE_LEANP):
+        o8, l8 = oracle.attn_fp8_emul(q, k, v, mode=mode, T=8)
+        o5, l5 = oracle.attn_fp8_emul(q, k, v, mode=mode, T=5)
+        assert np.allclose(o8, o5, atol=1e-14) and np.allclose(l8, l5, atol=1e-13)
+
+
+def test_emul_lse_consistent_with_rounded_weights():
+    # lse_emul - lse_exact = ln(sum p~ 2^e / sum 2^y): within the rounding
+    # error band (exact mode: |.| <= ln(1+1/16); Lean P: [ln(2^-1/16), ln(1.0615*2^1/16)])
+    q, k, v = (t.numpy() for t in workloads.make_custom(1, 256, 256, 2, 2, 64, 16, seed=20))
+    _, l = oracle.attn_ref(q, k, v)
+    _, le = oracle.attn_fp8_emul(q, k, v, mode=oracle.MODE_EXACT)
+    assert np.all(np.abs(le - l) <= np.log(1 + 1 / 16))
+    _, ll = oracle.attn_fp8_emul(q, k, v, mode=oracle.MODE_LEANP)
+    assert np.all(ll - l >= np.log(2.0 ** (-1 / 16)) - 1e-12)
+    assert np.all(ll - l <= np.log(1.0615 * 2.0 ** (1 / 16)))
+
+
+# ----------------------------------------------------- tolerance feasibility
+@pytest.mark.parametrize("mode,tol", [(oracle.MODE_EXACT, 4e-2), (oracle.MODE_LEANP, 6e-2)])
+def test_fp8_emulation_meets_tolerance_on_tiny(mode, tol):
+    w = workloads.get("tiny")
+    q, k, v = (t.numpy() for t in workloads.make_inputs(w))
+    cq, dq = oracle.quantize_fp8(q)
+    ck, dk = oracle.quantize_fp8(k)
+    cv, dv = oracle.quantize_fp8(v)
+    qd, kd, vd = oracle.dequant_e4m3(cq, dq), oracle.dequant_e4m3(ck, dk), oracle.dequant_e4m3(cv, dv)
+    o, _ = oracle.attn_ref(qd, kd, vd)
+    oe, _ = oracle.attn_fp8_emul(qd, kd, vd, mode=mode)
+    err = oracle.rel_rmse(oe, o)
+    assert err <= tol, err
