@@ -1,0 +1,227 @@
+"""B200 (sm_100a) causal prefill attention in FP8 e4m3 and BF16.
+
+A thin ctypes binding over ``libzattn.so`` (the C ABI in ``include/zattn.h``).
+Every step of the computation runs in this package's CUDA kernels; PyTorch is
+only used for device memory and streams.  There is no CPU fallback: if the
+shared library is missing, importing this package raises.
+
+Low-level names mirror the C ABI (``zq_attn_fwd``, ``zq_attn_fwd_ex``,
+``zq_quantize_fp8``, ...) and take raw integers (device addresses, sizes, a
+stream handle).  The torch-level helpers ``attn_fwd``, ``quantize_fp8`` and
+``flash_attn_func`` marshal tensors into those calls.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import re
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libzattn.so")
+HEADER_PATH = os.path.join(os.path.dirname(HERE), "include", "zattn.h")
+
+ZQ_DTYPE_BF16, ZQ_DTYPE_FP8_E4M3 = 0, 1
+ZQ_X_F32, ZQ_X_BF16 = 0, 1
+ZQ_SOFTMAX_EXACT, ZQ_SOFTMAX_LEANP = 0, 1
+ZQ_OK, ZQ_ERR_NULL, ZQ_ERR_SHAPE, ZQ_ERR_UNSUPPORTED = 0, -1, -2, -3
+ZQ_ERR_ALIGN, ZQ_ERR_ARCH, ZQ_ERR_CUDA, ZQ_ERR_TIMEOUT = -4, -5, -6, -7
+
+
+class ZQError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__("%s failed: %s (%d)" % (where, zq_status_string(status), status))
+        self.status = status
+
+
+class zq_attn_args(ctypes.Structure):
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+        ("out", ctypes.c_void_p), ("lse", ctypes.c_void_p),
+        ("B", ctypes.c_int), ("Sq", ctypes.c_int), ("Sk", ctypes.c_int), ("Hq", ctypes.c_int),
+        ("Hkv", ctypes.c_int), ("d_qk", ctypes.c_int), ("d_v", ctypes.c_int),
+        ("softmax_scale", ctypes.c_float), ("causal", ctypes.c_int), ("dtype", ctypes.c_int),
+        ("q_descale", ctypes.c_void_p), ("k_descale", ctypes.c_void_p), ("v_descale", ctypes.c_void_p),
+        ("softmax_mode", ctypes.c_int), ("block_scale", ctypes.c_int), ("headroom_T", ctypes.c_int),
+        ("status", ctypes.c_void_p),
+    ]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            "libzattn.so not found at %s; build it with `python bf16_causal_prefill_02_b200/build.py`"
+            % LIB_PATH
+        )
+    lib = ctypes.CDLL(LIB_PATH)
+    P, i32, i64, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float
+    lib.zq_attn_fwd.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32, f32, i32, i32,
+                                P, P, P, P]
+    lib.zq_attn_fwd.restype = i32
+    lib.zq_attn_fwd_ex.argtypes = [ctypes.POINTER(zq_attn_args), P]
+    lib.zq_attn_fwd_ex.restype = i32
+    lib.zq_attn_fwd_debug.argtypes = [ctypes.POINTER(zq_attn_args), P, P]
+    lib.zq_attn_fwd_debug.restype = i32
+    lib.zq_quantize_fp8.argtypes = [P, i32, i64, i32, i32, P, P, P, P]
+    lib.zq_quantize_fp8.restype = i32
+    lib.zq_quantize_workspace_bytes.argtypes = []
+    lib.zq_quantize_workspace_bytes.restype = ctypes.c_size_t
+    lib.zq_status_string.argtypes = [i32]
+    lib.zq_status_string.restype = ctypes.c_char_p
+    lib.zq_version.argtypes = []
+    lib.zq_version.restype = i32
+    return lib
+
+
+_lib = _load()
+
+
+def header_functions() -> list[str]:
+    """Names of the functions include/zattn.h declares."""
+    txt = open(HEADER_PATH).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(zq_[a-z0-9_]+)\s*\(", txt)))
+
+
+# ------------------------------------------------------------------ C ABI names
+def zq_attn_fwd(q, k, v, out, lse, B, Sq, Sk, Hq, Hkv, d_qk, d_v, softmax_scale, causal, dtype,
+                q_descale, k_descale, v_descale, stream) -> int:
+    return _lib.zq_attn_fwd(q, k, v, out, lse, B, Sq, Sk, Hq, Hkv, d_qk, d_v, softmax_scale,
+                            causal, dtype, q_descale, k_descale, v_descale, stream)
+
+
+def zq_attn_fwd_ex(args: zq_attn_args, stream) -> int:
+    return _lib.zq_attn_fwd_ex(ctypes.byref(args), stream)
+
+
+def zq_attn_fwd_debug(args: zq_attn_args, dbg, stream) -> int:
+    return _lib.zq_attn_fwd_debug(ctypes.byref(args), dbg, stream)
+
+
+ZQ_DEBUG_BYTES = 128 * 128 * 4 + 128 * 64 * 4 + 128 * 4
+
+
+def zq_quantize_fp8(x, x_dtype, n_vec, d, hadamard, x_fp8, descale, workspace, stream) -> int:
+    return _lib.zq_quantize_fp8(x, x_dtype, n_vec, d, hadamard, x_fp8, descale, workspace, stream)
+
+
+def zq_quantize_workspace_bytes() -> int:
+    return int(_lib.zq_quantize_workspace_bytes())
+
+
+def zq_status_string(status: int) -> str:
+    return _lib.zq_status_string(status).decode()
+
+
+def zq_version() -> int:
+    return int(_lib.zq_version())
+
+
+# ------------------------------------------------------------- torch helpers
+def _torch():
+    import torch
+
+    return torch
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream):
+    torch = _torch()
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _check(rc: int, where: str):
+    if rc != ZQ_OK:
+        raise ZQError(rc, where)
+
+
+def _is_fp8(t) -> bool:
+    torch = _torch()
+    return t.dtype in (torch.float8_e4m3fn, torch.uint8)
+
+
+def quantize_fp8(x, hadamard: bool = False, out=None, descale=None, workspace=None, stream=None):
+    """Per-tensor e4m3 quantisation of a CUDA tensor (fp32 or bf16, last dim d).
+
+    Returns (codes as torch.float8_e4m3fn, descale fp32 tensor of shape (1,))."""
+    torch = _torch()
+    if not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous CUDA tensor")
+    if x.dtype == torch.float32:
+        xd = ZQ_X_F32
+    elif x.dtype == torch.bfloat16:
+        xd = ZQ_X_BF16
+    else:
+        raise TypeError("quantize_fp8 takes float32 or bfloat16")
+    d = x.shape[-1]
+    if out is None:
+        out = torch.empty(x.shape, dtype=torch.float8_e4m3fn, device=x.device)
+    if descale is None:
+        descale = torch.empty(1, dtype=torch.float32, device=x.device)
+    if workspace is None:
+        workspace = torch.empty(zq_quantize_workspace_bytes(), dtype=torch.uint8, device=x.device)
+    _check(zq_quantize_fp8(x.data_ptr(), xd, x.numel() // d, d, int(bool(hadamard)), out.data_ptr(),
+                           descale.data_ptr(), workspace.data_ptr(), _stream(stream)), "zq_quantize_fp8")
+    return out, descale
+
+
+def attn_fwd(q, k, v, out=None, lse=None, softmax_scale=None, causal=True, q_descale=None,
+             k_descale=None, v_descale=None, softmax_mode=ZQ_SOFTMAX_LEANP, block_scale=True,
+             headroom_T=8, status=None, return_lse=True, stream=None, debug=None):
+    """Causal prefill attention on CUDA tensors.
+
+    q (B,Sq,Hq,d_qk), k (B,Sk,Hkv,d_qk), v (B,Sk,Hkv,d_v): bfloat16, or FP8
+    e4m3 (float8_e4m3fn / uint8) with per-tensor fp32 descale tensors.
+    Returns (out bf16 (B,Sq,Hq,d_v), lse fp32 (B,Hq,Sq) or None)."""
+    torch = _torch()
+    for t in (q, k, v):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous CUDA tensors")
+    if _is_fp8(q) and _is_fp8(k) and _is_fp8(v):
+        dtype = ZQ_DTYPE_FP8_E4M3
+    elif q.dtype == k.dtype == v.dtype == torch.bfloat16:
+        dtype = ZQ_DTYPE_BF16
+    else:
+        raise TypeError("q, k, v must all be bfloat16 or all FP8 e4m3")
+    B, Sq, Hq, dqk = q.shape
+    Sk, Hkv, dv = k.shape[1], k.shape[2], v.shape[3]
+    if out is None:
+        out = torch.empty((B, Sq, Hq, dv), dtype=torch.bfloat16, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    a = zq_attn_args()
+    a.q, a.k, a.v, a.out, a.lse = q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), _ptr(lse)
+    a.B, a.Sq, a.Sk, a.Hq, a.Hkv, a.d_qk, a.d_v = B, Sq, Sk, Hq, Hkv, dqk, dv
+    a.softmax_scale = float(softmax_scale) if softmax_scale else 0.0
+    a.causal = int(bool(causal))
+    a.dtype = dtype
+    a.q_descale, a.k_descale, a.v_descale = _ptr(q_descale), _ptr(k_descale), _ptr(v_descale)
+    a.softmax_mode = int(softmax_mode)
+    a.block_scale = int(bool(block_scale))
+    a.headroom_T = int(headroom_T)
+    a.status = _ptr(status)
+    if debug is not None:
+        _check(zq_attn_fwd_debug(a, debug.data_ptr(), _stream(stream)), "zq_attn_fwd_debug")
+    else:
+        _check(zq_attn_fwd_ex(a, _stream(stream)), "zq_attn_fwd_ex")
+    return out, lse
+
+
+def flash_attn_func(q, k, v, softmax_scale=None, causal=True, return_attn_probs=False, **fp8_kwargs):
+    """flash_attn_func-style entry: (B,S,H,d) tensors in, (B,S,H,d_v) bf16 out.
+
+    With return_attn_probs=True returns (out, lse, None) like flash-attn."""
+    out, lse = attn_fwd(q, k, v, softmax_scale=softmax_scale, causal=causal,
+                        return_lse=return_attn_probs, **fp8_kwargs)
+    return (out, lse, None) if return_attn_probs else out
+
+
+def causal_flops(B, Sq, Hq, dqk, dv, Sk=None) -> float:
+    """2*B*Hq*S^2*(d_qk+d_v)/2 for the causal Sq == Sk case."""
+    S = Sq if Sk is None else math.sqrt(Sq * Sk)
+    return 2.0 * B * Hq * S * S * (dqk + dv) / 2.0

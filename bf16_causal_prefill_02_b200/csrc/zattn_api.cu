@@ -1,0 +1,177 @@
+// zattn_api.cu -- the C ABI declared in include/zattn.h: argument
+// validation, device checks and kernel launches.  No allocation, no
+// synchronisation, no state kept between calls.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "../../include/zattn.h"
+
+#include "zq_internal.h"
+
+namespace {
+
+constexpr int kVersion = 100;  // 0.1.0
+constexpr uint64_t kTimeoutNs = 2000000000ull;  // bound on any single device-side wait
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Current device must be sm_100 (B200 class).  Returns the SM count through
+// `num_sms` when non-null.
+int check_device(int* num_sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ZQ_ERR_CUDA;
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return ZQ_ERR_CUDA;
+  if (major != 10 || minor != 0) return ZQ_ERR_ARCH;
+  if (num_sms &&
+      cudaDeviceGetAttribute(num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return ZQ_ERR_CUDA;
+  return ZQ_OK;
+}
+
+int validate_attn(const zq_attn_args* a) {
+  if (!a) return ZQ_ERR_NULL;
+  if (!a->q || !a->k || !a->v || !a->out) return ZQ_ERR_NULL;
+  if (a->B <= 0 || a->Sq <= 0 || a->Sk <= 0 || a->Hq <= 0 || a->Hkv <= 0) return ZQ_ERR_SHAPE;
+  if (a->Hq % a->Hkv != 0) return ZQ_ERR_SHAPE;
+  if (!((a->d_qk == 128 && a->d_v == 128) || (a->d_qk == 192 && a->d_v == 128)))
+    return ZQ_ERR_UNSUPPORTED;
+  if (a->dtype != ZQ_DTYPE_BF16 && a->dtype != ZQ_DTYPE_FP8_E4M3) return ZQ_ERR_UNSUPPORTED;
+  if (a->dtype == ZQ_DTYPE_FP8_E4M3) {
+    if (a->softmax_mode != ZQ_SOFTMAX_EXACT && a->softmax_mode != ZQ_SOFTMAX_LEANP)
+      return ZQ_ERR_UNSUPPORTED;
+    if (a->block_scale != 0 && a->block_scale != 1) return ZQ_ERR_UNSUPPORTED;
+    if (a->headroom_T < 0 || a->headroom_T > 8) return ZQ_ERR_UNSUPPORTED;
+  }
+  if (!(std::isfinite(a->softmax_scale))) return ZQ_ERR_SHAPE;
+  // grid = n_qtiles * B * Hq blocks; TMA element counts and strides
+  const int64_t ntiles = (a->Sq + 127) / 128;
+  if (ntiles * a->B * (int64_t)a->Hq > 0x7FFFFFFFll) return ZQ_ERR_SHAPE;
+  const int es = a->dtype == ZQ_DTYPE_BF16 ? 2 : 1;
+  const int64_t qbytes = (int64_t)a->B * a->Sq * a->Hq * a->d_qk * es;
+  const int64_t kbytes = (int64_t)a->B * a->Sk * a->Hkv * a->d_qk * es;
+  if (qbytes >= (1ll << 40) || kbytes >= (1ll << 40)) return ZQ_ERR_SHAPE;
+  if (!aligned16(a->q) || !aligned16(a->k) || !aligned16(a->v) || !aligned16(a->out) ||
+      (a->lse && !aligned16(a->lse)))
+    return ZQ_ERR_ALIGN;
+  return ZQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int zq_version(void) { return kVersion; }
+
+const char* zq_status_string(int s) {
+  switch (s) {
+    case ZQ_OK: return "ok";
+    case ZQ_ERR_NULL: return "a required pointer is NULL";
+    case ZQ_ERR_SHAPE: return "invalid shape (size <= 0, Hq % Hkv != 0 or too large)";
+    case ZQ_ERR_UNSUPPORTED: return "unsupported head dims, dtype, mode or option";
+    case ZQ_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case ZQ_ERR_ARCH: return "current device is not sm_100 (B200)";
+    case ZQ_ERR_CUDA: return "CUDA call failed";
+    case ZQ_ERR_TIMEOUT: return "a device-side wait timed out";
+    default: return "unknown status";
+  }
+}
+
+static int attn_impl(const zq_attn_args* a, void* dbg, void* stream) {
+  int rc = validate_attn(a);
+  if (rc != ZQ_OK) return rc;
+  rc = check_device(nullptr);
+  if (rc != ZQ_OK) return rc;
+  zq::AttnLaunch L;
+  L.q = a->q;
+  L.k = a->k;
+  L.v = a->v;
+  L.dqk = a->d_qk;
+  L.dv = a->d_v;
+  L.dtype = a->dtype;
+  L.mode = a->softmax_mode;
+  L.block_scale = a->block_scale;
+  L.p.out = a->out;
+  L.p.lse = a->lse;
+  L.p.q_descale = a->q_descale;
+  L.p.k_descale = a->k_descale;
+  L.p.v_descale = a->v_descale;
+  L.p.status = a->status;
+  L.p.B = a->B;
+  L.p.Sq = a->Sq;
+  L.p.Sk = a->Sk;
+  L.p.Hq = a->Hq;
+  L.p.Hkv = a->Hkv;
+  L.p.n_qtiles = (a->Sq + 127) / 128;
+  L.p.causal = a->causal ? 1 : 0;
+  L.p.headroom_T = a->dtype == ZQ_DTYPE_FP8_E4M3 ? a->headroom_T : 8;
+  L.p.softmax_scale =
+      a->softmax_scale > 0.0f ? a->softmax_scale : (float)(1.0 / std::sqrt((double)a->d_qk));
+  L.p.timeout_ns = kTimeoutNs;
+  L.p.dbg = dbg;
+  cudaError_t e = zq::launch_attention(L, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ZQ_OK : ZQ_ERR_CUDA;
+}
+
+int zq_attn_fwd_ex(const zq_attn_args* a, void* stream) { return attn_impl(a, nullptr, stream); }
+
+int zq_attn_fwd_debug(const zq_attn_args* a, void* dbg, void* stream) {
+  if (!dbg) return ZQ_ERR_NULL;
+  return attn_impl(a, dbg, stream);
+}
+
+int zq_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B,
+                int Sq, int Sk, int Hq, int Hkv, int d_qk, int d_v, float softmax_scale,
+                int causal, int dtype, const float* q_descale, const float* k_descale,
+                const float* v_descale, void* stream) {
+  zq_attn_args a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.out = out;
+  a.lse = lse;
+  a.B = B;
+  a.Sq = Sq;
+  a.Sk = Sk;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.d_qk = d_qk;
+  a.d_v = d_v;
+  a.softmax_scale = softmax_scale;
+  a.causal = causal;
+  a.dtype = dtype;
+  a.q_descale = q_descale;
+  a.k_descale = k_descale;
+  a.v_descale = v_descale;
+  a.softmax_mode = ZQ_SOFTMAX_LEANP;
+  a.block_scale = 1;
+  a.headroom_T = 8;
+  a.status = nullptr;
+  return zq_attn_fwd_ex(&a, stream);
+}
+
+size_t zq_quantize_workspace_bytes(void) { return 256; }
+
+int zq_quantize_fp8(const void* x, int x_dtype, int64_t n_vec, int d, int hadamard,
+                    void* x_fp8, float* descale, void* workspace, void* stream) {
+  if (!x || !x_fp8 || !descale || !workspace) return ZQ_ERR_NULL;
+  if (n_vec < 0 || d <= 0) return ZQ_ERR_SHAPE;
+  if (x_dtype != ZQ_X_F32 && x_dtype != ZQ_X_BF16) return ZQ_ERR_UNSUPPORTED;
+  if (d % 8 != 0 || (hadamard && d % 128 != 0)) return ZQ_ERR_UNSUPPORTED;
+  if (n_vec > (int64_t)1 << 40 || n_vec * (int64_t)d > ((int64_t)1 << 40)) return ZQ_ERR_SHAPE;
+  if (!aligned16(x) || !aligned16(x_fp8) || !aligned16(workspace)) return ZQ_ERR_ALIGN;
+  int sms = 0;
+  int rc = check_device(&sms);
+  if (rc != ZQ_OK) return rc;
+  cudaError_t e = zq::launch_quantize(x, x_dtype == ZQ_X_BF16, n_vec * (int64_t)d,
+                                      hadamard ? 1 : 0, x_fp8, descale, workspace,
+                                      static_cast<cudaStream_t>(stream), sms);
+  return e == cudaSuccess ? ZQ_OK : ZQ_ERR_CUDA;
+}
+
+}  // extern "C"

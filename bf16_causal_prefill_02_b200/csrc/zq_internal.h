@@ -1,0 +1,41 @@
+// zq_internal.h -- launch structures shared by the C-ABI layer and the
+// kernels (internal; not part of the public interface).
+#pragma once
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace zq {
+
+struct AttnParams {
+  void* out;  // (B, Sq, Hq, d_v) bfloat16
+  float* lse;  // (B, Hq, Sq) or nullptr
+  const float* q_descale;
+  const float* k_descale;
+  const float* v_descale;
+  int* status;
+  int B, Sq, Sk, Hq, Hkv;
+  int n_qtiles;
+  int causal;
+  int headroom_T;
+  float softmax_scale;
+  uint64_t timeout_ns;
+  // Debug dump (nullptr in normal use): the CTA of (batch 0, head 0, query
+  // tile 0) writes its first score tile, P words and scale words here:
+  // float S[128][128]; uint32 P[128][64]; uint32 SF[128].
+  void* dbg;
+};
+
+struct AttnLaunch {
+  const void* q;
+  const void* k;
+  const void* v;
+  AttnParams p;
+  int dqk, dv, dtype, mode, block_scale;
+};
+
+cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t st);
+cudaError_t launch_quantize(const void* x, int x_bf16, int64_t n, int hadamard, void* out,
+                            float* descale, void* workspace, cudaStream_t st, int num_sms);
+
+}  // namespace zq

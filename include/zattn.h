@@ -1,0 +1,177 @@
+/*
+ * zattn.h -- C ABI of the B200 (sm_100a) causal prefill attention library.
+ *
+ * Operations follow the ZYFA announcement as re-reported by three web pages:
+ *   [P1] "Zyphra ZYFA : FlashAttention en FP8 pour l'AMD MI355X, jusqu'a
+ *        1,76 fois plus rapide" (lefilia.fr), paragraphs 1-3.
+ *   [P2] "Zyphra rilascia ZYFA, kernel di attenzione FP8 ottimizzati per le
+ *        GPU AMD" (aicronaca.it), sections "Che cosa ha annunciato Zyphra"
+ *        and "Perche l'FP8 non basta da solo".
+ *   [P3] "Zyphra ZYFA ... FP8 FlashAttention for AMD MI355X up to 1.76x"
+ *        (ai4bro.com), sections TL;DR and "How ZYFA works".
+ *
+ * Conventions shared by every entry point
+ *   - Pointers named q, k, v, out, lse, x, x_fp8, descale, workspace and
+ *     status are DEVICE pointers on the current CUDA device; the caller owns
+ *     all of them.  The library allocates nothing and keeps no state between
+ *     calls (it is safe to call from several host threads).
+ *   - `stream` is a cudaStream_t passed as void*; NULL is the legacy default
+ *     stream.  Every call is asynchronous on that stream and never
+ *     synchronises.
+ *   - Return value: ZQ_OK (0) or a negative ZQ_ERR_* code.  On an argument
+ *     error nothing is launched and no output is written.  ZQ_ERR_CUDA means
+ *     a launch failed (cudaGetLastError is left set for the caller).
+ */
+#ifndef ZATTN_H_
+#define ZATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ZQ_API __attribute__((visibility("default")))
+#else
+#define ZQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- element types ---- */
+#define ZQ_DTYPE_BF16 0      /* q, k, v bfloat16 */
+#define ZQ_DTYPE_FP8_E4M3 1  /* q, k, v OCP e4m3fn bytes with fp32 descales */
+
+#define ZQ_X_F32 0  /* quantiser input fp32 */
+#define ZQ_X_BF16 1 /* quantiser input bfloat16 */
+
+/* ---- FP8 softmax modes ---- */
+#define ZQ_SOFTMAX_EXACT 0 /* P~ = e4m3_rne(exp2(y - e))                   */
+#define ZQ_SOFTMAX_LEANP 1 /* P~ bits = clamp(rne(8 (y - e)) + 56, 0, 126) */
+
+/* ---- status codes ---- */
+#define ZQ_OK 0
+#define ZQ_ERR_NULL (-1)        /* a required pointer is NULL              */
+#define ZQ_ERR_SHAPE (-2)       /* a size <= 0, Hq % Hkv != 0, overflow    */
+#define ZQ_ERR_UNSUPPORTED (-3) /* head dims, dtype, mode or option        */
+#define ZQ_ERR_ALIGN (-4)       /* a pointer is not 16-byte aligned        */
+#define ZQ_ERR_ARCH (-5)        /* current device is not sm_100            */
+#define ZQ_ERR_CUDA (-6)        /* a CUDA driver/runtime call failed       */
+#define ZQ_ERR_TIMEOUT (-7)     /* a device-side wait ran out (status word) */
+
+/*
+ * zq_attn_fwd -- causal (or full) forward prefill attention,
+ *   out = softmax(q k^T * softmax_scale + mask) v,  lse = logsumexp per row.
+ * [P3 TL;DR: causal forward (prefill) attention in FP8 e4m3 and BF16, head
+ *  dim 128 and the MLA 192/128 shape; P2 "Che cosa ha annunciato Zyphra":
+ *  a drop-in for flash_attn_func.]
+ *
+ *   q    (B, Sq, Hq,  d_qk) contiguous, bf16 or e4m3 bytes
+ *   k    (B, Sk, Hkv, d_qk) contiguous, same type
+ *   v    (B, Sk, Hkv, d_v)  contiguous, same type
+ *   out  (B, Sq, Hq,  d_v)  contiguous bfloat16 (both input types)
+ *   lse  (B, Hq, Sq) fp32 natural log, or NULL to skip
+ *   (d_qk, d_v) in {(128,128), (192,128)};  Hq % Hkv == 0, query head h
+ *   reads kv head h / (Hq / Hkv) (GQA).
+ *   softmax_scale <= 0 selects 1/sqrt(d_qk).
+ *   causal != 0: key c is visible to query i iff c <= i + Sk - Sq
+ *   (bottom-right alignment); a query row with no visible key gets out = 0,
+ *   lse = -inf.
+ *   q/k/v_descale: device pointers to one fp32 each (per-tensor dequant
+ *   scale, FP8 only; NULL means 1.0); ignored for bf16.
+ *   FP8 uses Lean P with per-(row, 64-key block) power-of-2 scaling and
+ *   headroom 8 (see zq_attn_fwd_ex for the other modes).
+ * Errors: ZQ_ERR_NULL (q, k, v or out NULL), ZQ_ERR_SHAPE, ZQ_ERR_UNSUPPORTED,
+ *   ZQ_ERR_ALIGN (q, k, v, out, lse not 16-byte aligned), ZQ_ERR_ARCH,
+ *   ZQ_ERR_CUDA.
+ */
+ZQ_API int zq_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B,
+                int Sq, int Sk, int Hq, int Hkv, int d_qk, int d_v, float softmax_scale,
+                int causal, int dtype, const float* q_descale, const float* k_descale,
+                const float* v_descale, void* stream);
+
+/* Extended arguments for zq_attn_fwd_ex.  Fields up to v_descale have the
+ * meaning given for zq_attn_fwd. */
+typedef struct zq_attn_args {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* out;
+  float* lse;
+  int B, Sq, Sk, Hq, Hkv, d_qk, d_v;
+  float softmax_scale;
+  int causal;
+  int dtype;
+  const float* q_descale;
+  const float* k_descale;
+  const float* v_descale;
+  /* FP8 only.  softmax_mode: ZQ_SOFTMAX_EXACT or ZQ_SOFTMAX_LEANP
+   * [P1 paragraph 3, P2 "Perche l'FP8 non basta da solo": Lean P replaces the
+   * exponential by a multiply-add whose result is read as e4m3 bits]. */
+  int softmax_mode;
+  /* FP8 only.  1: every 64-key block of a row gets its own power-of-2
+   * exponent e = ceil(block max of y) - headroom_T, absorbed by the block-
+   * scaled PV matrix instruction [P1 paragraph 3; P3 "How ZYFA works" item
+   * 3].  0: one running exponent per row (ceil of the running max minus
+   * headroom_T), shared by all blocks. */
+  int block_scale;
+  /* FP8 only, 0..8: where the block maximum lands, 2^(T-1) < p~max <= 2^T. */
+  int headroom_T;
+  /* Optional device int.  Must hold 0 before the call; a device-side wait
+   * that runs out writes ZQ_ERR_TIMEOUT there and the kernel returns early
+   * (outputs are then undefined).  NULL: not reported. */
+  int* status;
+} zq_attn_args;
+
+/* zq_attn_fwd_ex -- zq_attn_fwd with the options above.  Same errors, plus
+ * ZQ_ERR_UNSUPPORTED for softmax_mode / block_scale / headroom_T out of
+ * range (they are ignored, not checked, for bf16). */
+ZQ_API int zq_attn_fwd_ex(const zq_attn_args* args, void* stream);
+
+/* zq_attn_fwd_debug -- zq_attn_fwd_ex that also dumps, for (batch 0,
+ * head 0, query tile 0), the first 128x128 score tile before masking and the
+ * P words written for it, to the device buffer `dbg` (caller-owned,
+ * ZQ_DEBUG_BYTES bytes): float S[128][128] (raw q.k dot products, no
+ * scale), uint32 P[128][64] (bf16: 64 words of 2 x bf16; FP8: the first 32
+ * words hold 4 x e4m3 each, key order little-endian), uint32 SF[128] (FP8:
+ * UE8M0 scale bytes of the four 32-key chunks of each row).  For tests. */
+#define ZQ_DEBUG_BYTES (128 * 128 * 4 + 128 * 64 * 4 + 128 * 4)
+ZQ_API int zq_attn_fwd_debug(const zq_attn_args* args, void* dbg, void* stream);
+
+/*
+ * zq_quantize_fp8 -- per-tensor FP8 e4m3 quantiser with an optional fused
+ * 128-point Walsh-Hadamard rotation [P2 "Perche l'FP8 non basta da solo":
+ * a Hadamard rotation of Q and K roughly halves the input quantisation error].
+ *
+ *   x        n_vec vectors of d channels, fp32 (x_dtype ZQ_X_F32) or bf16
+ *   hadamard != 0: every 128-channel slice is replaced by H_128 x (Sylvester
+ *            order, entries +-1, fp32 butterflies at strides 1,2,...,64);
+ *            requires d % 128 == 0.
+ *   amax     = max |x| (after rotation);  inv = fl32(448 / amax)
+ *   x_fp8    (n_vec, d) e4m3 bytes = e4m3_rne_satfinite(fl32(x * inv))
+ *   descale  one fp32 = fl32(amax / 448), times fl32(2^-3.5) when rotated,
+ *            so that (H q)(H k)^T descales to q k^T.  amax == 0 gives all-
+ *            zero codes and descale 0.
+ *   workspace  device scratch of zq_quantize_workspace_bytes() bytes, 16-byte
+ *            aligned; its contents on entry do not matter and it must not be
+ *            used by another call that runs at the same time.
+ * Errors: ZQ_ERR_NULL, ZQ_ERR_SHAPE (n_vec < 0, d <= 0), ZQ_ERR_UNSUPPORTED
+ *   (x_dtype, hadamard with d % 128 != 0, d % 8 != 0), ZQ_ERR_ALIGN (x,
+ *   x_fp8, workspace not 16-byte aligned), ZQ_ERR_ARCH, ZQ_ERR_CUDA.
+ */
+ZQ_API int zq_quantize_fp8(const void* x, int x_dtype, int64_t n_vec, int d, int hadamard,
+                    void* x_fp8, float* descale, void* workspace, void* stream);
+
+/* Bytes of device scratch zq_quantize_fp8 needs (a small constant). */
+ZQ_API size_t zq_quantize_workspace_bytes(void);
+
+/* Static text for a status code (never NULL). */
+ZQ_API const char* zq_status_string(int status);
+
+/* Library version as major*10000 + minor*100 + patch. */
+ZQ_API int zq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ZATTN_H_ */

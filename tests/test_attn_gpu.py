@@ -1,0 +1,172 @@
+"""GPU parity of the attention kernels against the oracle (element by element
+at small sizes, sampled rows at the benchmark sizes), plus determinism and the
+debug dumps that isolate QK^T and the P generation."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from attn_cases import Case, check_against_oracle
+
+pytestmark = pytest.mark.gpu
+
+DTYPES = ["bf16", "exact", "leanp"]
+
+
+def _debug_run(case):
+    import bf16_causal_prefill_02_b200 as zq
+
+    dbg = torch.zeros(zq.ZQ_DEBUG_BYTES // 4, dtype=torch.float32, device="cuda")
+    o, l = case.run_gpu(debug=dbg)
+    torch.cuda.synchronize()
+    d = dbg.cpu()
+    S = d[: 128 * 128].numpy().reshape(128, 128).astype(np.float64)
+    P = d[128 * 128 : 128 * 128 + 128 * 64].view(torch.int32).numpy().view(np.uint32).reshape(128, 64)
+    SF = d[128 * 128 + 128 * 64 :].view(torch.int32).numpy().view(np.uint32)
+    return o, l, S, P, SF
+
+
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("dqk", [128, 192])
+def test_debug_score_tile_is_qk(dtype, dqk):
+    c = Case(1, 128, 128, 1, 1, dqk, 128, dtype=dtype, seed=1)
+    _, _, S, _, _ = _debug_run(c)
+    if c.fp8:
+        qv = oracle.e4m3_decode(c.cq[0, :, 0])
+        kv = oracle.e4m3_decode(c.ck[0, :, 0])
+    else:
+        qv, kv = c.qd[0, :, 0], c.kd[0, :, 0]
+    ref = qv @ kv.T
+    err = np.abs(S - ref).max() / np.abs(ref).max()
+    assert err < 1e-5, err
+
+
+def test_debug_leanp_codes_match_emulation():
+    c = Case(1, 128, 128, 1, 1, 128, 128, dtype="leanp", seed=2)
+    _, _, S, P, SF = _debug_run(c)
+    codes = P[:, :32].copy().view(np.uint8).reshape(128, 128)
+    match = total = 0
+    for r in (0, 1, 31, 63, 64, 100, 127):
+        _, _, p = oracle.attn_fp8_emul(c.qd, c.kd, c.vd, mode=oracle.MODE_LEANP, rows=[r], want_p=True)
+        got = oracle.e4m3_decode(codes[r, : r + 1])
+        match += int(np.sum(got == p[: r + 1]))
+        total += r + 1
+        assert np.all(codes[r, r + 1 :] == 0)  # masked keys
+    assert match / total >= 0.995, (match, total)
+
+
+def test_debug_exact_codes_match_emulation():
+    c = Case(1, 128, 128, 1, 1, 128, 128, dtype="exact", seed=3)
+    _, _, S, P, SF = _debug_run(c)
+    codes = P[:, :32].copy().view(np.uint8).reshape(128, 128)
+    match = total = 0
+    for r in (0, 5, 64, 90, 127):
+        _, _, p = oracle.attn_fp8_emul(c.qd, c.kd, c.vd, mode=oracle.MODE_EXACT, rows=[r], want_p=True)
+        got = oracle.e4m3_decode(codes[r, : r + 1])
+        match += int(np.sum(got == p[: r + 1]))
+        total += r + 1
+    assert match / total >= 0.995, (match, total)
+
+
+@pytest.mark.parametrize("dtype", DTYPES)
+def test_tiny_workload(dtype):
+    w = workloads.get("tiny")
+    c = Case(w.B, w.S, w.S, w.Hq, w.Hkv, w.dqk, w.dv, dtype=dtype, inputs=workloads.make_inputs(w))
+    check_against_oracle(c)
+
+
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("S", [1, 2, 127, 129, 300, 1000])
+def test_ragged_lengths(dtype, S):
+    check_against_oracle(Case(1, S, S, 2, 1, 128, 128, dtype=dtype, seed=S))
+
+
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("Sq,Sk", [(100, 300), (300, 100), (128, 256), (1, 500), (257, 129)])
+def test_unequal_lengths_bottom_right(dtype, Sq, Sk):
+    check_against_oracle(Case(1, Sq, Sk, 2, 2, 128, 128, dtype=dtype, seed=Sq + Sk))
+
+
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("Hq,Hkv", [(8, 2), (4, 1), (3, 3)])
+def test_gqa_mapping(dtype, Hq, Hkv):
+    check_against_oracle(Case(2, 200, 200, Hq, Hkv, 128, 128, dtype=dtype, seed=Hq * 10 + Hkv))
+
+
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("Sq,Sk", [(200, 200), (64, 300)])
+def test_non_causal(dtype, Sq, Sk):
+    check_against_oracle(Case(1, Sq, Sk, 2, 1, 128, 128, dtype=dtype, causal=False, seed=5))
+
+
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("S", [300, 640])
+def test_mla_192_128(dtype, S):
+    check_against_oracle(Case(1, S, S, 2, 2, 192, 128, dtype=dtype, seed=S))
+
+
+@pytest.mark.parametrize("dtype", ["exact", "leanp"])
+@pytest.mark.parametrize("T", [0, 4, 8])
+@pytest.mark.parametrize("block_scale", [True, False])
+def test_fp8_options(dtype, T, block_scale):
+    check_against_oracle(Case(1, 700, 700, 2, 1, 128, 128, dtype=dtype, T=T, block_scale=block_scale,
+                              seed=T, std=1.5))
+
+
+@pytest.mark.parametrize("dtype", ["exact", "leanp"])
+def test_fp8_hadamard_rotated_inputs(dtype):
+    w = workloads.get("long")
+    inputs = workloads.make_custom(1, 512, 512, 4, 2, 128, 128, seed=11)
+    q, k, v = inputs
+    q[..., [3, 40, 77, 120]] *= 20.0
+    k[..., [9, 50, 60, 101]] *= 20.0
+    c = Case(1, 512, 512, 4, 2, 128, 128, dtype=dtype, hadamard=True, inputs=(q, k, v))
+    check_against_oracle(c)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "leanp"])
+def test_large_logits_lazy_rescale(dtype):
+    # scores growing along the sequence force the reference max / exponent
+    # to move many times
+    q, k, v = workloads.make_custom(1, 600, 600, 2, 2, 128, 128, seed=21)
+    ramp = torch.linspace(0.2, 6.0, 600)[None, :, None, None]
+    check_against_oracle(Case(1, 600, 600, 2, 2, 128, 128, dtype=dtype, inputs=(q * 3.0, k * ramp, v)))
+
+
+@pytest.mark.parametrize("dtype", DTYPES)
+def test_bitwise_deterministic(dtype):
+    c = Case(1, 1000, 1000, 4, 2, 128, 128, dtype=dtype, seed=7)
+    o0, l0 = c.run_gpu()
+    for _ in range(20):
+        o, l = c.run_gpu(out=torch.empty_like(o0), lse=torch.empty_like(l0))
+        assert torch.equal(o.view(torch.int16), o0.view(torch.int16))
+        assert torch.equal(l.view(torch.int32), l0.view(torch.int32))
+
+
+def test_status_word_stays_zero():
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    c = Case(1, 256, 256, 2, 2, 128, 128, dtype="leanp", seed=1)
+    c.run_gpu(status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+
+
+# ---------------------------------------------------------------- full size
+FULL = [
+    ("gqa", "bf16", False), ("gqa", "leanp", False), ("gqa", "exact", False),
+    ("long", "leanp", False), ("long", "exact", False), ("long", "leanp", True), ("long", "exact", True),
+    ("mla", "bf16", False), ("mla", "leanp", False), ("mla", "exact", False),
+    ("gauss", "bf16", False), ("gauss", "leanp", False), ("gauss", "exact", False),
+]
+
+
+@pytest.mark.parametrize("name,dtype,had", FULL)
+def test_full_size_sampled_rows(name, dtype, had):
+    w = workloads.get(name)
+    c = Case(w.B, w.S, w.S, w.Hq, w.Hkv, w.dqk, w.dv, dtype=dtype, hadamard=had,
+             inputs=workloads.make_inputs(w))
+    every = max(64, w.S // 32)
+    rows = workloads.sample_rows(w.B, w.Hq, w.S, every=every).numpy()
+    res = check_against_oracle(c, rows=rows)
+    print(name, dtype, had, res)

@@ -1,0 +1,111 @@
+"""C-ABI boundary checks that need no GPU: the library loads, exports every
+function include/zattn.h declares, and rejects bad arguments with the
+documented status before touching the device.
+
+No test here passes a fake pointer together with otherwise valid arguments,
+so nothing can reach a kernel launch on a machine that has a GPU.
+"""
+import ctypes
+
+import pytest
+
+import bf16_causal_prefill_02_b200 as zq
+
+
+def test_library_exports_every_header_function():
+    names = zq.header_functions()
+    assert set(names) >= {"zq_attn_fwd", "zq_attn_fwd_ex", "zq_quantize_fp8",
+                          "zq_quantize_workspace_bytes", "zq_status_string", "zq_version"}
+    lib = ctypes.CDLL(zq.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings_and_version():
+    for s in range(0, -8, -1):
+        assert zq.zq_status_string(s) and zq.zq_status_string(s) != "unknown status"
+    assert zq.zq_status_string(-99) == "unknown status"
+    assert zq.zq_version() >= 100
+    assert zq.zq_quantize_workspace_bytes() >= 4
+
+
+A = 1 << 20  # a 16-byte aligned address that is never dereferenced
+
+
+def _args(**kw):
+    a = zq.zq_attn_args()
+    d = dict(q=A, k=A, v=A, out=A, lse=None, B=1, Sq=128, Sk=128, Hq=2, Hkv=1, d_qk=128, d_v=128,
+             softmax_scale=0.0, causal=1, dtype=zq.ZQ_DTYPE_BF16, q_descale=None, k_descale=None,
+             v_descale=None, softmax_mode=zq.ZQ_SOFTMAX_LEANP, block_scale=1, headroom_T=8, status=None)
+    d.update(kw)
+    for k, v in d.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), zq.ZQ_ERR_NULL),
+    (dict(k=None), zq.ZQ_ERR_NULL),
+    (dict(v=None), zq.ZQ_ERR_NULL),
+    (dict(out=None), zq.ZQ_ERR_NULL),
+    (dict(B=0), zq.ZQ_ERR_SHAPE),
+    (dict(Sq=-1), zq.ZQ_ERR_SHAPE),
+    (dict(Sk=0), zq.ZQ_ERR_SHAPE),
+    (dict(Hq=3, Hkv=2), zq.ZQ_ERR_SHAPE),
+    (dict(Hkv=0), zq.ZQ_ERR_SHAPE),
+    (dict(d_qk=64, d_v=64), zq.ZQ_ERR_UNSUPPORTED),
+    (dict(d_qk=128, d_v=192), zq.ZQ_ERR_UNSUPPORTED),
+    (dict(d_qk=256, d_v=128), zq.ZQ_ERR_UNSUPPORTED),
+    (dict(dtype=2), zq.ZQ_ERR_UNSUPPORTED),
+    (dict(dtype=1, softmax_mode=2), zq.ZQ_ERR_UNSUPPORTED),
+    (dict(dtype=1, block_scale=2), zq.ZQ_ERR_UNSUPPORTED),
+    (dict(dtype=1, headroom_T=9), zq.ZQ_ERR_UNSUPPORTED),
+    (dict(dtype=1, headroom_T=-1), zq.ZQ_ERR_UNSUPPORTED),
+    (dict(q=A + 8), zq.ZQ_ERR_ALIGN),
+    (dict(out=A + 2), zq.ZQ_ERR_ALIGN),
+    (dict(lse=A + 4), zq.ZQ_ERR_ALIGN),
+    (dict(softmax_scale=float("nan")), zq.ZQ_ERR_SHAPE),
+    (dict(B=65536, Sq=1 << 20, Hq=64, Hkv=64), zq.ZQ_ERR_SHAPE),
+])
+def test_attn_argument_errors(kw, code):
+    assert zq.zq_attn_fwd_ex(_args(**kw), None) == code
+
+
+def test_attn_plain_entry_validates_too():
+    rc = zq.zq_attn_fwd(A, A, A, None, None, 1, 128, 128, 2, 1, 128, 128, 0.0, 1, 0, None, None, None, None)
+    assert rc == zq.ZQ_ERR_NULL
+    rc = zq.zq_attn_fwd(A, A, A, A, None, 1, 128, 128, 3, 2, 128, 128, 0.0, 1, 0, None, None, None, None)
+    assert rc == zq.ZQ_ERR_SHAPE
+
+
+@pytest.mark.parametrize("args,code", [
+    ((None, 0, 4, 128, 0, A, A, A), zq.ZQ_ERR_NULL),
+    ((A, 0, 4, 128, 0, None, A, A), zq.ZQ_ERR_NULL),
+    ((A, 0, 4, 128, 0, A, None, A), zq.ZQ_ERR_NULL),
+    ((A, 0, 4, 128, 0, A, A, None), zq.ZQ_ERR_NULL),
+    ((A, 0, -1, 128, 0, A, A, A), zq.ZQ_ERR_SHAPE),
+    ((A, 0, 4, 0, 0, A, A, A), zq.ZQ_ERR_SHAPE),
+    ((A, 2, 4, 128, 0, A, A, A), zq.ZQ_ERR_UNSUPPORTED),
+    ((A, 0, 4, 12, 0, A, A, A), zq.ZQ_ERR_UNSUPPORTED),
+    ((A, 0, 4, 192, 1, A, A, A), zq.ZQ_ERR_UNSUPPORTED),
+    ((A + 4, 0, 4, 128, 0, A, A, A), zq.ZQ_ERR_ALIGN),
+    ((A, 0, 4, 128, 0, A + 1, A, A), zq.ZQ_ERR_ALIGN),
+    ((A, 0, 4, 128, 0, A, A, A + 8), zq.ZQ_ERR_ALIGN),
+])
+def test_quantize_argument_errors(args, code):
+    x, xd, n, d, had, out, ds, ws = args
+    assert zq.zq_quantize_fp8(x, xd, n, d, had, out, ds, ws, None) == code
+
+
+def test_no_cpu_fallback_without_library(tmp_path, monkeypatch):
+    # The binding must fail loudly when the shared library is missing.
+    import importlib.util
+    import shutil
+
+    pkg = tmp_path / "zpkg"
+    pkg.mkdir()
+    shutil.copy(zq.__file__, pkg / "__init__.py")
+    spec = importlib.util.spec_from_file_location("zpkg", pkg / "__init__.py")
+    mod = importlib.util.module_from_spec(spec)
+    with pytest.raises(ImportError):
+        spec.loader.exec_module(mod)

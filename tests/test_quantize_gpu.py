@@ -1,0 +1,85 @@
+"""GPU parity of the FP8 quantiser against the oracle's quantiser: bitwise
+identical codes and descale, with and without the fused Hadamard rotation."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(x32: torch.Tensor, src: str, hadamard: bool):
+    import bf16_causal_prefill_02_b200 as zq
+
+    if src == "bf16":
+        xb = x32.to(torch.bfloat16)
+        ref_in = xb.view(torch.int16).numpy().view(np.uint16)
+        xg = xb.cuda()
+    else:
+        ref_in = x32.numpy()
+        xg = x32.cuda()
+    codes, ds = zq.quantize_fp8(xg, hadamard=hadamard)
+    torch.cuda.synchronize()
+    rc, rds = oracle.quantize_fp8(ref_in, hadamard=hadamard)
+    return codes.view(torch.uint8).cpu().numpy(), float(ds.cpu()[0]), rc, float(rds)
+
+
+@pytest.mark.parametrize("hadamard", [False, True])
+@pytest.mark.parametrize("src", ["f32", "bf16"])
+@pytest.mark.parametrize("n_vec,d", [(1000, 128), (1, 128), (4097, 256)])
+def test_quantize_bitwise(n_vec, d, src, hadamard):
+    x = torch.randn((n_vec, d), generator=torch.Generator().manual_seed(n_vec + d)) * 3.0
+    g, gds, r, rds = _run(x, src, hadamard)
+    assert gds == rds
+    assert np.array_equal(g, r), "%d of %d codes differ" % (int((g != r).sum()), g.size)
+
+
+@pytest.mark.parametrize("n_vec,d", [(333, 192), (5, 8), (7, 24)])
+def test_quantize_bitwise_other_widths(n_vec, d):
+    x = torch.randn((n_vec, d), generator=torch.Generator().manual_seed(d))
+    g, gds, r, rds = _run(x, "f32", False)
+    assert gds == rds and np.array_equal(g, r)
+
+
+def test_quantize_empty_and_zero():
+    import bf16_causal_prefill_02_b200 as zq
+
+    codes, ds = zq.quantize_fp8(torch.zeros((0, 128), device="cuda"))
+    torch.cuda.synchronize()
+    assert float(ds.cpu()[0]) == 0.0
+    codes, ds = zq.quantize_fp8(torch.zeros((64, 128), device="cuda"))
+    assert float(ds.cpu()[0]) == 0.0 and not codes.view(torch.uint8).any()
+
+
+def test_quantize_outliers_saturate_nothing():
+    x = torch.randn((512, 128), generator=torch.Generator().manual_seed(3))
+    x[7, 5] = 1e4
+    x[100, 64] = -3e4
+    g, gds, r, rds = _run(x, "f32", False)
+    assert gds == rds and np.array_equal(g, r)
+    assert g.reshape(-1)[100 * 128 + 64] == 0xFE
+
+
+@pytest.mark.parametrize("hadamard", [False, True])
+def test_quantize_full_size_q_at_32k(hadamard):
+    """The Gaussian 32K workload's Q (32768 x 32 heads x 128): the size the
+    benchmark quantises every step."""
+    w = workloads.get("gauss")
+    g = torch.Generator().manual_seed(w.seed)
+    x = torch.randn((w.B * w.S * w.Hq, w.dqk), generator=g)
+    gc, gds, rc, rds = _run(x, "f32", hadamard)
+    assert gds == rds
+    assert np.array_equal(gc, rc)
+
+
+def test_quantize_repeatable():
+    import bf16_causal_prefill_02_b200 as zq
+
+    x = torch.randn((2048, 128), generator=torch.Generator().manual_seed(9)).cuda()
+    outs = [zq.quantize_fp8(x, hadamard=True) for _ in range(5)]
+    torch.cuda.synchronize()
+    c0 = outs[0][0].view(torch.uint8)
+    for c, d in outs[1:]:
+        assert torch.equal(c.view(torch.uint8), c0) and torch.equal(d, outs[0][1])
