@@ -1,0 +1,430 @@
+"""Benchmark: causal prefill attention TFLOP/s on B200 (FP8 e4m3 / BF16).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--dtype leanp|exact|bf16] [--impl reference] [--sweep]
+
+A step is one pass of the whole hot path over one batch of synthetic input:
+for FP8, the per-tensor quantisation of Q, K and V (fp32 -> e4m3, three
+quantiser calls) followed by the attention kernel; for BF16 the attention
+kernel alone.  The headline workload is the Gaussian peak-sweep point at
+S = 32768 (B=1, Hq=Hkv=32, d=128), FP8 with Lean P and per-64-key block
+scaling -- the configuration the pages quote their best FP8 number on.
+
+value      causal TFLOP/s = 2*B*Hq*S^2*(d_qk+d_v)/2 / step time (inputs resident
+           in HBM), summed over ranks (weak scaling: every rank runs its own
+           batch of the same size).
+e2e        same metric through the C ABI from pinned host buffers: H2D copy of
+           fp32 Q/K/V, the step, D2H of the bf16 output, all inside the timed
+           region.
+roofline   attention kernel only: algorithmic FLOPs per launch / CUDA-event
+           launch time, against the dense tensor peak of its dtype.
+cpu_baseline  the fp64 oracle (FP8 emulation of the same mode) on host cores
+           over a bounded row sample, in the same unit.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+DATASHEET_DENSE_TFLOPS = {"bf16": 2250.0, "fp8": 4500.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=40)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="gauss")
+    ap.add_argument("--S", type=int, default=None)
+    ap.add_argument("--dtype", default="leanp", choices=["leanp", "exact", "bf16"])
+    ap.add_argument("--hadamard", action="store_true")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--sweep", action="store_true", help="also print one line per workload/dtype")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ helpers
+def dist_setup(n):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+                power.append(float(f[3]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        loaded = [s for s, p in zip(sm, power) if p > 300] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_max": max(power) if power else None}
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def tensor_peak(kind: str):
+    """Dense tensor peak for the attention kernel, TFLOP/s.  The kernel runs
+    back to back for the whole timed region, so the sustained cuBLAS BF16
+    figure is the reference; FP8 takes it times the nominal FP8:BF16 ratio 2."""
+    pk, src = measured_peaks()
+    base = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
+    if kind == "fp8":
+        return base * 2.0, "%s bf16 sustained x2 (nominal fp8:bf16 ratio)" % src
+    return base, "%s bf16 sustained" % src
+
+
+def load_traffic(key: str):
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    return d.get(key)
+
+
+# --------------------------------------------------------------- our arm
+class Step:
+    """The hot path for one workload on one GPU; inputs resident in HBM."""
+
+    def __init__(self, w: workloads.Workload, dtype: str, hadamard: bool, seed_offset: int = 0):
+        import bf16_causal_prefill_02_b200 as zq
+
+        self.zq, self.w, self.dtype, self.hadamard = zq, w, dtype, hadamard
+        q, k, v = workloads.make_inputs(w, seed=w.seed + seed_offset)
+        self.host = [t.pin_memory() for t in (q, k, v)]
+        dev = torch.device("cuda")
+        self.q32, self.k32, self.v32 = (t.to(dev) for t in self.host)
+        B, S, Hq, Hkv, dqk, dv = w.B, w.S, w.Hq, w.Hkv, w.dqk, w.dv
+        self.out = torch.empty((B, S, Hq, dv), dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty((B, Hq, S), dtype=torch.float32, device=dev)
+        self.out_host = torch.empty_like(self.out, device="cpu").pin_memory()
+        if dtype == "bf16":
+            self.qb, self.kb, self.vb = (t.to(torch.bfloat16) for t in (self.q32, self.k32, self.v32))
+        else:
+            f8 = torch.float8_e4m3fn
+            self.qc = torch.empty(self.q32.shape, dtype=f8, device=dev)
+            self.kc = torch.empty(self.k32.shape, dtype=f8, device=dev)
+            self.vc = torch.empty(self.v32.shape, dtype=f8, device=dev)
+            self.ds = torch.zeros(3, dtype=torch.float32, device=dev)
+            self.ws = torch.empty(3, zq.zq_quantize_workspace_bytes(), dtype=torch.uint8, device=dev)
+        self.mode = zq.ZQ_SOFTMAX_EXACT if dtype == "exact" else zq.ZQ_SOFTMAX_LEANP
+        self.ev = []
+
+    def launches_per_step(self) -> int:
+        return 1 if self.dtype == "bf16" else 7  # 3 x (amax + write) + attention
+
+    def attention(self, ev=None):
+        zq = self.zq
+        if ev is not None:
+            ev[0].record()
+        if self.dtype == "bf16":
+            zq.attn_fwd(self.qb, self.kb, self.vb, out=self.out, lse=self.lse)
+        else:
+            zq.attn_fwd(self.qc, self.kc, self.vc, out=self.out, lse=self.lse,
+                        q_descale=self.ds[0:1], k_descale=self.ds[1:2], v_descale=self.ds[2:3],
+                        softmax_mode=self.mode, block_scale=True, headroom_T=8)
+        if ev is not None:
+            ev[1].record()
+
+    def quantize(self):
+        zq = self.zq
+        zq.quantize_fp8(self.q32, hadamard=self.hadamard, out=self.qc, descale=self.ds[0:1], workspace=self.ws[0])
+        zq.quantize_fp8(self.k32, hadamard=self.hadamard, out=self.kc, descale=self.ds[1:2], workspace=self.ws[1])
+        zq.quantize_fp8(self.v32, hadamard=False, out=self.vc, descale=self.ds[2:3], workspace=self.ws[2])
+
+    def step(self, ev=None):
+        if self.dtype != "bf16":
+            self.quantize()
+        self.attention(ev)
+
+    def e2e_step(self):
+        """Host buffers in, host buffer out, through the same C-ABI calls."""
+        self.q32.copy_(self.host[0], non_blocking=True)
+        self.k32.copy_(self.host[1], non_blocking=True)
+        self.v32.copy_(self.host[2], non_blocking=True)
+        if self.dtype == "bf16":
+            self.qb.copy_(self.q32)
+            self.kb.copy_(self.k32)
+            self.vb.copy_(self.v32)
+        self.step()
+        self.out_host.copy_(self.out, non_blocking=True)
+
+    def h2d_bytes(self):
+        return sum(t.numel() * t.element_size() for t in self.host)
+
+    def d2h_bytes(self):
+        return self.out.numel() * self.out.element_size()
+
+
+def time_steps(fn, steps, warmup, world):
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    st = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(steps):
+        fn()
+    e1.record(st)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = e0.elapsed_time(e1)
+    return max_over_ranks(ms, world)
+
+
+def cpu_oracle_rate(w, dtype, seconds, hadamard=False):
+    """Time the oracle on host cores over a bounded row sample of `w`.
+    Returns (TFLOP/s, cores, sample description)."""
+    import oracle
+
+    q, k, v = (t.numpy() for t in workloads.make_inputs(w))
+    if dtype == "bf16":
+        qd, kd, vd = (torch.from_numpy(t).to(torch.bfloat16).double().numpy() for t in (q, k, v))
+    else:
+        deq = []
+        for t, rot in ((q, hadamard), (k, hadamard), (v, False)):
+            c, d = oracle.quantize_fp8(t, hadamard=rot)
+            deq.append(oracle.dequant_e4m3(c, float(d)))
+        qd, kd, vd = deq
+    S = w.S
+    rng = np.random.default_rng(0)
+    done_rows, flops, elapsed = 0, 0.0, 0.0
+    batch = 64
+    while elapsed < seconds:
+        rows = rng.integers(0, w.B * w.Hq * S, size=batch)
+        i = rows % S
+        t0 = time.perf_counter()
+        if dtype == "bf16":
+            oracle.attn_ref(qd, kd, vd, rows=rows)
+        else:
+            oracle.attn_fp8_emul(qd, kd, vd, rows=rows,
+                                 mode=oracle.MODE_EXACT if dtype == "exact" else oracle.MODE_LEANP)
+        elapsed += time.perf_counter() - t0
+        flops += float(np.sum(2.0 * (w.dqk + w.dv) * (i + 1)))
+        done_rows += batch
+        batch = min(batch * 2, 4096)
+    desc = ("%d uniformly drawn query rows of %s (fp64 %s on kernel inputs; inputs quantised "
+            "beforehand, untimed), %.1f s" % (done_rows, w.name,
+                                               "R1 exact" if dtype == "bf16" else "R2 " + dtype, elapsed))
+    return flops / elapsed / 1e12, oracle.num_threads(), desc
+
+
+def run_ours(args, rank, world, w):
+    import bf16_causal_prefill_02_b200 as zq  # noqa: F401  (fails loudly without the .so)
+
+    step = Step(w, args.dtype, args.hadamard, seed_offset=rank)
+    flops = w.causal_flops()
+    sampler = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
+    # warm-up + attention-only event timing for the roofline
+    for _ in range(max(args.warmup, 3)):
+        step.step()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.25)
+    ms_total = time_steps(step.step, args.steps, args.warmup, world)
+    # per-launch attention time on the launching stream
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    for e in evs:
+        step.step(e)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    attn_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    attn_ms = max_over_ranks(attn_ms, world)
+    ms_step = ms_total / args.steps
+    total_flops = sum_over_ranks(flops, world)
+    value = total_flops / (ms_step * 1e-3) / 1e12
+    # end to end from host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e_steps = max(3, min(args.steps, 10))
+        ms_e2e = time_steps(step.e2e_step, e2e_steps, 2, world) / e2e_steps
+        e2e = {"value": round(total_flops / (ms_e2e * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+               "ms_per_step": round(ms_e2e, 3),
+               "h2d_bytes_per_step": step.h2d_bytes(), "d2h_bytes_per_step": step.d2h_bytes()}
+    kind = "bf16" if args.dtype == "bf16" else "fp8"
+    peak, peak_src = tensor_peak(kind)
+    achieved = flops / (attn_ms * 1e-3) / 1e12
+    tkey = "%s_%s_S%d" % (w.name.split("_S")[0], args.dtype, w.S)
+    traffic = load_traffic(tkey)
+    res = {
+        "metric": "causal prefill attention TFLOP/s (FP8, BF16) at S=16K/32K; % of B200 tensor peak",
+        "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp8_e4m3" if kind == "fp8" else "bf16", "data": "synthetic",
+        "config": {"workload": "%s_%s%s" % (w.name, args.dtype, "_hadamard" if args.hadamard else ""),
+                   "B": w.B, "S": w.S, "Hq": w.Hq, "Hkv": w.Hkv, "d_qk": w.dqk, "d_v": w.dv,
+                   "causal": True, "softmax": args.dtype,
+                   "block_scale": kind == "fp8", "headroom_T": 8 if kind == "fp8" else None,
+                   "step": ("quantise Q,K,V (fp32->e4m3) + attention" if kind == "fp8" else "attention"),
+                   "l2": "inputs larger than L2 (%.0f MB fp32 Q/K/V), no flush" %
+                         (3 * w.B * w.S * w.Hq * w.dqk * 4 / 1e6),
+                   "parallelism": "dp%d (independent batches, no collective)" % world},
+        "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel", "achieved": round(achieved, 1),
+                     "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "peak_source": peak_src, "traffic": traffic,
+                     "frac_of_datasheet_dense": round(achieved / DATASHEET_DENSE_TFLOPS[kind], 4),
+                     "attn_ms": round(attn_ms, 4)},
+        "clocks": clocks,
+        "e2e": e2e,
+        "gpu_launches": step.launches_per_step() * args.steps,
+    }
+    return res
+
+
+def main():
+    args = parse()
+    rank, world, local = dist_setup(args.gpus)
+    w = workloads.get(args.workload, args.S)
+    if args.impl == "reference":
+        if rank == 0:
+            tf, cores, desc = cpu_oracle_rate(w, args.dtype, args.cpu_seconds * max(1, args.steps) / 40.0,
+                                              args.hadamard)
+            line = {"impl": "reference", "metric": "causal prefill attention TFLOP/s (FP8, BF16) at "
+                    "S=16K/32K; % of B200 tensor peak", "value": tf, "unit": "TFLOP/s",
+                    "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+                    "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                    "dtype": "f64", "data": "synthetic",
+                    "config": {"workload": "%s_%s" % (w.name, args.dtype)},
+                    "cpu_baseline": {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                                     "sample": desc},
+                    "e2e": {"value": tf, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                            "d2h_bytes_per_step": 0}}
+            print(json.dumps(line), flush=True)
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+        return
+    res = run_ours(args, rank, world, w)
+    if rank == 0 and not args.no_cpu:
+        tf, cores, desc = cpu_oracle_rate(w, args.dtype, args.cpu_seconds, args.hadamard)
+        res["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                               "sample": desc}
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if args.sweep and world == 1:
+        for name, S, dt in [("gauss", 4096, "leanp"), ("gauss", 8192, "leanp"), ("gauss", 16384, "leanp"),
+                            ("gauss", 32768, "exact"), ("gauss", 32768, "bf16"), ("gauss", 16384, "bf16"),
+                            ("mla", None, "leanp"), ("mla", None, "bf16"), ("long", None, "leanp"),
+                            ("gqa", None, "leanp"), ("gqa", None, "bf16")]:
+            a2 = argparse.Namespace(**vars(args))
+            a2.dtype, a2.no_e2e = dt, True
+            r = run_ours(a2, rank, world, workloads.get(name, S))
+            print(json.dumps({"sweep": r["config"]["workload"], "S": r["config"]["S"],
+                              "value": r["value"], "attn_tflops": r["roofline"]["achieved"],
+                              "frac": r["roofline"]["frac"], "ms_per_step": r["ms_per_step"],
+                              "attn_ms": r["roofline"]["attn_ms"], "clocks": r["clocks"]}), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

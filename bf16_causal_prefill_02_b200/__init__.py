@@ -98,7 +98,7 @@ def zq_attn_fwd_debug(args: zq_attn_args, dbg, stream) -> int:
     return _lib.zq_attn_fwd_debug(ctypes.byref(args), dbg, stream)
 
 
-ZQ_DEBUG_BYTES = 128 * 128 * 4 + 128 * 64 * 4 + 128 * 4
+ZQ_DEBUG_BYTES = 128 * 128 * 4 + 128 * 64 * 4 + 256 * 4
 
 
 def zq_quantize_fp8(x, x_dtype, n_vec, d, hadamard, x_fp8, descale, workspace, stream) -> int:

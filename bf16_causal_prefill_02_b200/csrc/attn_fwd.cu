@@ -16,16 +16,19 @@
 //        "How ZYFA works" (scaling by powers of 2 before rounding).
 //
 // One CTA computes one 128-row query tile of one (batch, head).  Warp roles:
-//   warps 0-3  softmax + epilogue; thread t owns query row t (TMEM lane t)
-//   warp 4     TMA producer (Q once, then K/V tiles through an NS-stage ring)
-//   warp 5     TMEM allocator and single-thread tcgen05.mma issuer
+//   warps 0-7  softmax + epilogue.  Warps w and w+4 share TMEM lane quarter
+//              w%4, so thread t (t < 256) owns query row t%128 and the half
+//              h = t/128 of every 128-key tile: keys [64h, 64h+64), which is
+//              exactly one 64-key scaling block.
+//   warp 8     TMA producer (Q once, then K/V tiles through an NS-stage ring)
+//   warp 9     TMEM allocator and single-thread tcgen05.mma issuer
 // Tensor memory (512 columns x 128 lanes, fp32 words):
 //   S0 [0,128) S1 [128,256)   score tiles; P (bf16x2 or 4 x e4m3 per word)
 //                             is written over the first columns of its S
 //   O  [256,256+DV)           output accumulator
 //   RS [384,400)              FP8: rounded row sum (P times a ones matrix)
-//   SFA0/SFA1 [400,404),[404,408)  FP8: per-(row, 32-key chunk) UE8M0 scales
-//   SFB [408,412)             FP8: scales of V / ones, all 2^0
+//   SFA [400,416)             FP8: UE8M0 scales of P, [buffer][half] x 4 cols
+//   SFB [416,420)             FP8: scales of V / ones, all 2^0
 // MMA issue order: QK_0, QK_1, PV_0, QK_2, PV_1, ... so the softmax of tile
 // j+1 overlaps PV_j and QK_{j+2}.
 #include <cuda_fp8.h>
@@ -40,9 +43,12 @@
 namespace zq {
 
 constexpr int kTile = 128;
-constexpr int kThreads = 192;
-constexpr uint32_t kColS0 = 0, kColO = 256, kColRS = 384, kColSFA = 400, kColSFB = 408;
+constexpr int kSoftmaxThreads = 256;
+constexpr int kThreads = kSoftmaxThreads + 64;
+constexpr int kWarpProducer = 8, kWarpMma = 9;
+constexpr uint32_t kColS0 = 0, kColO = 256, kColRS = 384, kColSFA = 400, kColSFB = 416;
 constexpr uint32_t kTmemCols = 512;
+constexpr int kInvalidExp = -(1 << 20);
 
 template <int DT, int DQK, int DV>
 struct Geo {
@@ -61,9 +67,11 @@ struct Geo {
   static constexpr int OFF_K = OFF_Q + QBYTES;
   static constexpr int OFF_V = OFF_K + NS * KBYTES;
   static constexpr int OFF_ONES = OFF_V + NS * VBYTES;     // 16 x 128 keys e4m3, K-major
-  static constexpr int OFF_SF = OFF_ONES + 2048;           // 2 x 128 uint32
-  static constexpr int OFF_BAR = OFF_SF + 1024;
-  static constexpr int NBAR = 1 + 4 * NS + 2 + 2 + 1 + 2 + 1;
+  static constexpr int OFF_X = OFF_ONES + 2048;            // exchange: [2 buf][2 half][128] int
+  static constexpr int OFF_XR = OFF_X + 2048;              // [2 buf][128] int (reference)
+  static constexpr int OFF_XL = OFF_XR + 1024;             // [2 half][128] float (row sums)
+  static constexpr int OFF_BAR = OFF_XL + 1024;
+  static constexpr int NBAR = 1 + 4 * NS + 2 + 2 + 1 + 1 + 2 + 1;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;  // + alignment slack
   static_assert(QBYTES % 1024 == 0 && VBYTES % 1024 == 0, "1 KB aligned tiles");
 };
@@ -78,6 +86,19 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
 }
+__device__ __forceinline__ float fma_sat(float a, float b, float c) {
+  float d;
+  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+// (a0, a1) * b + c on the paired fp32 FMA path
+__device__ __forceinline__ void ffma2(float& r0, float& r1, float a0, float a1, float b, float c) {
+  asm("{\n\t.reg .b64 x, y, z;\n\t"
+      "mov.b64 x, {%2, %3};\n\tmov.b64 y, {%4, %4};\n\tmov.b64 z, {%5, %5};\n\t"
+      "fma.rn.f32x2 x, x, y, z;\n\tmov.b64 {%0, %1}, x;\n\t}"
+      : "=f"(r0), "=f"(r1)
+      : "f"(a0), "f"(a1), "f"(b), "f"(c));
+}
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   uint32_t d;
   asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
@@ -87,20 +108,32 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
 }
+__device__ __forceinline__ uint32_t pack_e4m3x4(float p0, float p1, float p2, float p3) {
+  const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(p0, p1), __NV_SATFINITE, __NV_E4M3);
+  const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(p2, p3), __NV_SATFINITE, __NV_E4M3);
+  return lo | (hi << 16);
+}
 __device__ __forceinline__ float pow2i(int e) {  // exact 2^e for -126 <= e <= 127
   return __int_as_float((e + 127) << 23);
 }
-// max over n consecutive floats with 3-input max
-template <int N>
-__device__ __forceinline__ float rowmax(const float* s) {
-  float m0 = s[0], m1 = s[1];
+// Max of 64 floats with four independent 3-input max chains.
+__device__ __forceinline__ float max64(const float* s) {
+  float m0 = s[0], m1 = s[1], m2 = s[2], m3 = s[3];
 #pragma unroll
-  for (int c = 2; c + 3 < N; c += 4) {
+  for (int c = 4; c < 64; c += 8) {
     m0 = max3(m0, s[c], s[c + 1]);
     m1 = max3(m1, s[c + 2], s[c + 3]);
+    m2 = max3(m2, s[c + 4], s[c + 5]);
+    m3 = max3(m3, s[c + 6], s[c + 7]);
   }
-  m0 = max3(m0, s[N - 2], s[N - 1]);
-  return fmaxf(m0, m1);
+  return fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+}
+// Reference-exponent rule shared by both halves of a row (FP8): returns the
+// exponent E after seeing this tile's largest block exponent `emax`.
+__device__ __forceinline__ int next_ref(int eref_old, int emax, int thr) {
+  if (emax <= kInvalidExp) return eref_old;
+  if (eref_old <= kInvalidExp) return emax;
+  return emax > eref_old + thr ? emax : eref_old;
 }
 
 template <int DT, int DQK, int DV, int MODE, int BS>
@@ -125,11 +158,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   // after them) and PV_j cannot start before P_j, so exactly phases j-1 and
   // j are possible and the parity test is unambiguous.
   uint64_t* bar_pvdone = bar_pfull + 2;      // [1]
-  uint64_t* bar_sf = bar_pvdone + 1;         // [2]
-  uint64_t* bar_ofinal = bar_sf + 2;         // [1] last PV landed
+  uint64_t* bar_ofinal = bar_pvdone + 1;     // [1] last PV landed
+  uint64_t* bar_x = bar_ofinal + 1;          // [2] per-tile exchange between halves
+  uint64_t* bar_ep = bar_x + 2;              // [1] epilogue exchange
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + G::NBAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  uint32_t* sf_smem = reinterpret_cast<uint32_t*>(smem + G::OFF_SF);  // [2][128]
+  int* xch = reinterpret_cast<int*>(smem + G::OFF_X);      // [2][2][128]
+  int* xref = reinterpret_cast<int*>(smem + G::OFF_XR);    // [2][128]
+  float* xl = reinterpret_cast<float*>(smem + G::OFF_XL);  // [2][128]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -143,7 +179,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int q0 = t * kTile;
   const int q1 = min(q0 + kTile - 1, p.Sq - 1);
   const int shift = p.Sk - p.Sq;
-  int max_key = p.causal ? min(q1 + shift, p.Sk - 1) : p.Sk - 1;
+  const int max_key = p.causal ? min(q1 + shift, p.Sk - 1) : p.Sk - 1;
   const int n_kv = max_key < 0 ? 0 : max_key / kTile + 1;
   const int min_lim = p.causal ? min(q0 + shift, p.Sk - 1) : p.Sk - 1;
 
@@ -157,11 +193,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar_sfull + s, 1);
-      mbar_init(bar_pfull + s, 128);
-      mbar_init(bar_sf + s, 128);
+      mbar_init(bar_pfull + s, kSoftmaxThreads);
+      mbar_init(bar_x + s, kSoftmaxThreads);
     }
     mbar_init(bar_pvdone, 1);
     mbar_init(bar_ofinal, 1);
+    mbar_init(bar_ep, kSoftmaxThreads);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -170,11 +207,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = threadIdx.x; i < 512; i += kThreads) ones[i] = 0x38383838u;
     fence_proxy_async_smem();
   }
-  if (warp == 5) {
+  if (warp == kWarpMma) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == kWarpProducer && lane == 0) {
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
@@ -194,7 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (p.status) atomicExch(p.status, -7 /* ZQ_ERR_TIMEOUT */);
   };
 
-  if (warp == 4) {
+  if (warp == kWarpProducer) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && n_kv > 0) {
       uint8_t* sq = smem + G::OFF_Q;
@@ -225,7 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_4d(sv + c * 16384, &tmV, bar_vfull + s, c * 128 / G::ES, g, j * kTile, b);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && n_kv > 0) {
       const uint32_t sbase = smem_u32(smem);
@@ -271,16 +308,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t dv = smem_desc(vb + kk * 16 * 128, 16384, 1024, SW_128B);
             mma_f16_ts(tbase + kColO, aP + kk * 8, dv, idesc_pv_bf16, acc);
           } else {
-            // 32 keys per step = 8 columns of 4 x e4m3; scale byte kk
+            // 32 keys per step = 8 columns of 4 x e4m3.  Keys 32kk.. belong to
+            // half kk/2; its scale word sits in SFA[buf][kk/2], byte kk%2.
             const uint64_t dv = smem_desc(vb + kk * 32 * 128, 16384, 1024, SW_128B);
-            const uint32_t sfa =
-                (tbase + kColSFA + (j & 1) * 4) | ((uint32_t)kk << 30);
-            const uint32_t sfb = (tbase + kColSFB) | ((uint32_t)kk << 30);
-            mma_mxf8_ts(tbase + kColO, aP + kk * 8, dv, idesc_mx(1u, 128, DV, kk, kk), sfa, sfb,
+            const uint32_t sid = (uint32_t)(kk & 1);
+            const uint32_t sfa = (tbase + kColSFA + (j & 1) * 8 + (kk >> 1) * 4) | (sid << 30);
+            const uint32_t sfb = (tbase + kColSFB) | (sid << 30);
+            mma_mxf8_ts(tbase + kColO, aP + kk * 8, dv, idesc_mx(1u, 128, DV, sid, sid), sfa, sfb,
                         acc);
-            const uint64_t d1 =
-                smem_desc(sbase + G::OFF_ONES + kk * 32, 16, 1024, SW_128B);
-            mma_mxf8_ts(tbase + kColRS, aP + kk * 8, d1, idesc_mx(0u, 128, 16, kk, kk), sfa,
+            const uint64_t d1 = smem_desc(sbase + G::OFF_ONES + kk * 32, 16, 1024, SW_128B);
+            mma_mxf8_ts(tbase + kColRS, aP + kk * 8, d1, idesc_mx(0u, 128, 16, sid, sid), sfa,
                         sfb, acc);
           }
         }
@@ -300,10 +337,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------ softmax (rows)
-    const int row = threadIdx.x;  // 0..127 == TMEM lane
+    const int half = threadIdx.x >> 7;  // which 64-key block of each tile
+    const int row = threadIdx.x & 127;  // query row == TMEM lane
+    const int quarter = warp & 3;
     const int i = q0 + row;
     const int row_lim = p.causal ? min(i + shift, p.Sk - 1) : p.Sk - 1;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const uint32_t col_h = (uint32_t)half * 64;  // first S / O column of this half
     float c = p.softmax_scale * 1.4426950408889634f;  // log2(e)
     float vscale = 1.0f;
     if (DT == 1) {
@@ -311,15 +351,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float kd = p.k_descale ? *p.k_descale : 1.0f;
       vscale = p.v_descale ? *p.v_descale : 1.0f;
       c = ((p.softmax_scale * qd) * kd) * 1.4426950408889634f;
-      // SFB (scales of V and of the ones matrix): all 2^0 = 0x7F
-      tmem_st4(tbase + lane_off + kColSFB, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+      if (half == 0) {
+        // SFB (scales of V and of the ones matrix): all 2^0 = 0x7F
+        tmem_st4(tbase + lane_off + kColSFB, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+      } else if (!BS) {
+        // running mode: every block scale is 2^0 as well
+        tmem_st4(tbase + lane_off + kColSFA, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+        tmem_st4(tbase + lane_off + kColSFA + 4, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+        tmem_st4(tbase + lane_off + kColSFA + 8, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+        tmem_st4(tbase + lane_off + kColSFA + 12, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+      }
       tmem_st_wait();
     }
     const int T = p.headroom_T;
-    float yref = -INFINITY;  // BF16: log2-domain reference max
-    int eref = 0;            // FP8: reference exponent E
-    bool have_ref = false;
-    float l = 0.0f;          // BF16 row sum (fp32, unrounded p)
+    float yref = -INFINITY;   // BF16 / FP8 running mode: log2-domain reference
+    int eref = kInvalidExp;   // FP8: reference exponent E (invalid until a key is seen)
+    float l = 0.0f;           // BF16 partial row sum over this half (fp32, unrounded p)
     bool ok = true;
 
     for (int j = 0; ok && j < n_kv; ++j) {
@@ -327,37 +374,41 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool w = mbar_wait(bar_sfull + buf, (j >> 1) & 1, lim, abort_flag);
       if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
       tc_fence_after();
-      uint32_t sr[128];
+      uint32_t sr[64];
       {
         uint32_t(&a0)[32] = *reinterpret_cast<uint32_t(*)[32]>(sr);
         uint32_t(&a1)[32] = *reinterpret_cast<uint32_t(*)[32]>(sr + 32);
-        uint32_t(&a2)[32] = *reinterpret_cast<uint32_t(*)[32]>(sr + 64);
-        uint32_t(&a3)[32] = *reinterpret_cast<uint32_t(*)[32]>(sr + 96);
-        const uint32_t ts = tbase + lane_off + kColS0 + buf * 128;
+        const uint32_t ts = tbase + lane_off + kColS0 + buf * 128 + col_h;
         tmem_ld32(ts, a0);
         tmem_ld32(ts + 32, a1);
-        tmem_ld32(ts + 64, a2);
-        tmem_ld32(ts + 96, a3);
         tmem_ld_wait();
       }
       float* s = reinterpret_cast<float*>(sr);
       const bool dump = p.dbg != nullptr && j == 0 && t == 0 && bh == 0;
       if (dump) {
-        float* ds = static_cast<float*>(p.dbg) + row * 128;
+        float* ds = static_cast<float*>(p.dbg) + row * 128 + col_h;
 #pragma unroll
-        for (int cc = 0; cc < 128; ++cc) ds[cc] = s[cc];
+        for (int cc = 0; cc < 64; ++cc) ds[cc] = s[cc];
       }
-      const int kbase = j * kTile;
-      if (kbase + kTile - 1 > min_lim) {
+      const int kbase = j * kTile + (int)col_h;
+      if (kbase + 63 > min_lim) {
 #pragma unroll
-        for (int cc = 0; cc < 128; ++cc)
+        for (int cc = 0; cc < 64; ++cc)
           if (kbase + cc > row_lim) s[cc] = -INFINITY;
       }
-      const uint32_t tP = tbase + lane_off + kColS0 + buf * 128;
+      const float m = max64(s);  // raw block maximum (scores before scaling)
+      int* xb = xch + buf * 256;
+      int* xr = xref + buf * 128;
 
       if constexpr (DT == 0) {
         // ------------------------------------------------ BF16, exact exp2
-        const float ymax = rowmax<128>(s) * c;
+        xb[half * 128 + row] = __float_as_int(m);
+        tc_fence_before();  // both halves' S loads complete before any P store
+        mbar_arrive(bar_x + buf);
+        w = mbar_wait(bar_x + buf, (j >> 1) & 1, lim, abort_flag);
+        if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+        tc_fence_after();
+        const float ymax = fmaxf(m, __int_as_float(xb[(half ^ 1) * 128 + row])) * c;
         const bool need = ymax > yref + 8.0f;
         if (__any_sync(0xffffffffu, need)) {
           const float nref = fmaxf(yref, ymax);
@@ -370,9 +421,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
             tc_fence_after();
 #pragma unroll 1
-            for (int ch = 0; ch < DV / 32; ++ch) {
+            for (int ch = 0; ch < 2; ++ch) {
               uint32_t o[32];
-              const uint32_t to = tbase + lane_off + kColO + ch * 32;
+              const uint32_t to = tbase + lane_off + kColO + col_h + ch * 32;
               tmem_ld32(to, o);
               tmem_ld_wait();
 #pragma unroll
@@ -382,125 +433,131 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         const float nb = yref == -INFINITY ? 0.0f : -yref;
-        uint32_t pk[64];
+        uint32_t pk[32];
+        float lp0 = 0.0f, lp1 = 0.0f;
 #pragma unroll
-        for (int cc = 0; cc < 128; cc += 2) {
-          const float p0 = ex2_approx(fmaf(s[cc], c, nb));
-          const float p1 = ex2_approx(fmaf(s[cc + 1], c, nb));
-          l += p0 + p1;
+        for (int cc = 0; cc < 64; cc += 2) {
+          float z0, z1;
+          ffma2(z0, z1, s[cc], s[cc + 1], c, nb);
+          const float p0 = ex2_approx(z0);
+          const float p1 = ex2_approx(z1);
+          lp0 += p0;
+          lp1 += p1;
           pk[cc / 2] = pack_bf16x2(p0, p1);
         }
-        tmem_st32(tP, *reinterpret_cast<uint32_t(*)[32]>(pk));
-        tmem_st32(tP + 32, *reinterpret_cast<uint32_t(*)[32]>(pk + 32));
+        l += lp0 + lp1;
+        tmem_st32(tbase + lane_off + kColS0 + buf * 128 + half * 32, pk);
         if (dump) {
           uint32_t* dp = reinterpret_cast<uint32_t*>(static_cast<float*>(p.dbg) + 128 * 128);
 #pragma unroll
-          for (int e = 0; e < 64; ++e) dp[row * 64 + e] = pk[e];
+          for (int e = 0; e < 32; ++e) dp[row * 64 + half * 32 + e] = pk[e];
         }
       } else {
         // ------------------------------------------------ FP8 P path
-        const float m0 = rowmax<64>(s), m1 = rowmax<64>(s + 64);
-        int e0, e1, emax;
-        bool v0, v1;
+        int e;  // this half's block exponent
         if (BS) {
-          v0 = m0 != -INFINITY;
-          v1 = m1 != -INFINITY;
-          e0 = v0 ? (int)ceilf(m0 * c) - T : -100000;
-          e1 = v1 ? (int)ceilf(m1 * c) - T : -100000;
-          emax = max(e0, e1);
+          e = m != -INFINITY ? (int)ceilf(m * c) - T : kInvalidExp;
+          xb[half * 128 + row] = e;
+          if (half == 0) xr[row] = eref;
         } else {
-          // running mode: one exponent from the running max, shared by both blocks
-          const float mm = fmaxf(m0, m1);
-          const float ymx = fmaxf(mm * c, yref);
-          yref = ymx;
-          v0 = v1 = ymx != -INFINITY;
-          e0 = e1 = emax = v0 ? (int)ceilf(ymx) - T : -100000;
+          xb[half * 128 + row] = __float_as_int(m);
         }
-        const bool valid = v0 || v1;
-        // reference exponent: first valid tile; raised lazily (block mode,
-        // when a block exceeds E by 32) or whenever it grows (running mode)
-        const bool need = valid && (!have_ref || emax > eref + (BS ? 32 : 0));
-        if (__any_sync(0xffffffffu, need)) {
-          const int nref = need ? emax : eref;
-          const float f = (have_ref && need) ? pow2i(max(eref - nref, -126)) : 1.0f;
-          const bool had = have_ref;
-          if (need) { eref = nref; have_ref = true; }
-          if (j > 0 && __any_sync(0xffffffffu, had && need)) {
-            w = mbar_wait(bar_pvdone, (j - 1) & 1, lim, abort_flag);
-            if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
-            tc_fence_after();
+        tc_fence_before();  // both halves' S loads complete before any P store
+        mbar_arrive(bar_x + buf);
+        w = mbar_wait(bar_x + buf, (j >> 1) & 1, lim, abort_flag);
+        if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+        tc_fence_after();
+        int nref;
+        if (BS) {
+          nref = next_ref(eref, max(e, xb[(half ^ 1) * 128 + row]), 32);
+        } else {
+          // running mode: one exponent from the running max of the row
+          const float mm = fmaxf(m, __int_as_float(xb[(half ^ 1) * 128 + row]));
+          yref = fmaxf(mm * c, yref);
+          nref = yref != -INFINITY ? (int)ceilf(yref) - T : kInvalidExp;
+          e = nref;
+        }
+        const bool had = eref > kInvalidExp;
+        const bool grow = had && nref != eref;
+        if (j > 0 && __any_sync(0xffffffffu, grow)) {
+          // O and the row sum hold tiles < j at scale 2^(-eref): move them to
+          // 2^(-nref) exactly.  PV_{j-1} must have landed first.
+          const float f = grow ? pow2i(max(eref - nref, -126)) : 1.0f;
+          w = mbar_wait(bar_pvdone, (j - 1) & 1, lim, abort_flag);
+          if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+          tc_fence_after();
 #pragma unroll 1
-            for (int ch = 0; ch < DV / 32; ++ch) {
-              uint32_t o[32];
-              const uint32_t to = tbase + lane_off + kColO + ch * 32;
-              tmem_ld32(to, o);
-              tmem_ld_wait();
+          for (int ch = 0; ch < 2; ++ch) {
+            uint32_t o[32];
+            const uint32_t to = tbase + lane_off + kColO + col_h + ch * 32;
+            tmem_ld32(to, o);
+            tmem_ld_wait();
 #pragma unroll
-              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
-              tmem_st32(to, o);
-            }
+            for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * f);
+            tmem_st32(to, o);
+          }
+          if (half == 0) {
             uint32_t rs;
             tmem_ld1(tbase + lane_off + kColRS, rs);
             tmem_ld_wait();
             tmem_st1(tbase + lane_off + kColRS, __float_as_uint(__uint_as_float(rs) * f));
           }
         }
-        // UE8M0 scale bytes 2^(e_k - E): chunks 0,1 -> block 0; 2,3 -> block 1
-        const int sf0 = v0 ? min(max(e0 - eref + 127, 0), 254) : 0;
-        const int sf1 = v1 ? min(max(e1 - eref + 127, 0), 254) : 0;
-        const uint32_t sfw = (uint32_t)sf0 * 0x0101u | ((uint32_t)sf1 * 0x0101u) << 16;
-        uint32_t pk[32];
+        eref = nref;
+        const bool valid = e > kInvalidExp;
+        uint32_t pk[16];
         if (MODE == 0) {
           // exact: e4m3_rne(exp2(y - e))
+          const float ne = valid ? -(float)e : 0.0f;
 #pragma unroll
-          for (int blk = 0; blk < 2; ++blk) {
-            const float ne = -(float)(blk == 0 ? (v0 ? e0 : 0) : (v1 ? e1 : 0));
-#pragma unroll
-            for (int cc = blk * 64; cc < blk * 64 + 64; cc += 4) {
-              const float p0 = ex2_approx(fmaf(s[cc], c, ne));
-              const float p1 = ex2_approx(fmaf(s[cc + 1], c, ne));
-              const float p2 = ex2_approx(fmaf(s[cc + 2], c, ne));
-              const float p3 = ex2_approx(fmaf(s[cc + 3], c, ne));
-              const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(p0, p1), __NV_SATFINITE, __NV_E4M3);
-              const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(p2, p3), __NV_SATFINITE, __NV_E4M3);
-              pk[cc / 4] = lo | (hi << 16);
-            }
+          for (int cc = 0; cc < 64; cc += 4) {
+            float z0, z1, z2, z3;
+            ffma2(z0, z1, s[cc], s[cc + 1], c, ne);
+            ffma2(z2, z3, s[cc + 2], s[cc + 3], c, ne);
+            pk[cc / 4] = pack_e4m3x4(ex2_approx(z0), ex2_approx(z1), ex2_approx(z2), ex2_approx(z3));
           }
         } else {
-          // Lean P: bits of fma(s, 8c, 56 - 8e + 1.5*2^23) hold rne(8(y-e))+56
-          // in their low byte; clamp at code 0 by an integer max.
-          const float c8 = c * 8.0f;
-          const int magic = 0x4B400000;  // bits of 1.5 * 2^23
+          // Lean P: u = sat((8(y - e) + 56) / 128) clamps the code at 0; the
+          // magic add 1.5*2^23 rounds 128u half-to-even into the low byte.
+          const float a = c * 0.0625f;                         // 8c / 128
+          const float k0 = valid ? (float)(56 - 8 * e) * 0.0078125f : 0.0f;
+          const float magic = 12582912.0f;
 #pragma unroll
-          for (int blk = 0; blk < 2; ++blk) {
-            const int e = blk == 0 ? (v0 ? e0 : 0) : (v1 ? e1 : 0);
-            const float kadd = 12582912.0f + (float)(56 - 8 * e);
-#pragma unroll
-            for (int cc = blk * 64; cc < blk * 64 + 64; cc += 4) {
-              const int b0 = max(__float_as_int(fmaf(s[cc], c8, kadd)), magic);
-              const int b1 = max(__float_as_int(fmaf(s[cc + 1], c8, kadd)), magic);
-              const int b2 = max(__float_as_int(fmaf(s[cc + 2], c8, kadd)), magic);
-              const int b3 = max(__float_as_int(fmaf(s[cc + 3], c8, kadd)), magic);
-              pk[cc / 4] = prmt(prmt(b0, b1, 0x0040u), prmt(b2, b3, 0x0040u), 0x5410u);
-            }
+          for (int cc = 0; cc < 64; cc += 4) {
+            const float u0 = fma_sat(s[cc], a, k0);
+            const float u1 = fma_sat(s[cc + 1], a, k0);
+            const float u2 = fma_sat(s[cc + 2], a, k0);
+            const float u3 = fma_sat(s[cc + 3], a, k0);
+            float x0, x1, x2, x3;
+            ffma2(x0, x1, u0, u1, 128.0f, magic);
+            ffma2(x2, x3, u2, u3, 128.0f, magic);
+            pk[cc / 4] = prmt(prmt(__float_as_uint(x0), __float_as_uint(x1), 0x0040u),
+                              prmt(__float_as_uint(x2), __float_as_uint(x3), 0x0040u), 0x5410u);
           }
         }
-        tmem_st32(tP, pk);
+        tmem_st16(tbase + lane_off + kColS0 + buf * 128 + half * 16, pk);
+        if (BS) {
+          // scale words for the four rows this thread's lane serves in the
+          // replicated SFA layout: column r/32 holds row r at lanes r%32+32q
+          uint32_t sw[4];
+#pragma unroll
+          for (int m1 = 0; m1 < 4; ++m1) {
+            const int rr = lane + 32 * m1;
+            const int ea = xb[rr], eb = xb[128 + rr];
+            const int en = next_ref(xr[rr], max(ea, eb), 32);
+            const int eo = half == 0 ? ea : eb;
+            const int sf = eo > kInvalidExp ? min(max(eo - en + 127, 0), 254) : 0;
+            sw[m1] = (uint32_t)sf * 0x01010101u;
+          }
+          tmem_st4(tbase + lane_off + kColSFA + buf * 8 + half * 4, sw[0], sw[1], sw[2], sw[3]);
+        }
         if (dump) {
           uint32_t* dp = reinterpret_cast<uint32_t*>(static_cast<float*>(p.dbg) + 128 * 128);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) dp[row * 64 + e] = pk[e];
-          dp[128 * 64 + row] = sfw;
+          for (int q = 0; q < 16; ++q) dp[row * 64 + half * 16 + q] = pk[q];
+          dp[128 * 64 + half * 128 + row] =
+              valid ? (uint32_t)min(max(e - eref + 127, 0), 254) * 0x01010101u : 0u;
         }
-        // scale factors: the row of query r goes to column r/32 of the SFA
-        // block, replicated in all four lane quarters (lane r%32 + 32q)
-        sf_smem[buf * 128 + row] = sfw;
-        mbar_arrive(bar_sf + buf);
-        w = mbar_wait(bar_sf + buf, (j >> 1) & 1, lim, abort_flag);
-        if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
-        tmem_st4(tbase + lane_off + kColSFA + buf * 4, sf_smem[buf * 128 + lane],
-                 sf_smem[buf * 128 + 32 + lane], sf_smem[buf * 128 + 64 + lane],
-                 sf_smem[buf * 128 + 96 + lane]);
       }
       tmem_st_wait();
       tc_fence_before();
@@ -510,11 +567,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       fail();
     } else {
       // ------------------------------------------------------------ epilogue
-      float L = l, lse_v = -INFINITY;
       bool wok = true;
       if (n_kv > 0) {
         wok = mbar_wait(bar_ofinal, 0, lim, abort_flag);
         wok = __all_sync(0xffffffffu, wok);
+      }
+      float L = 0.0f;
+      if (wok) {
+        if (DT == 0) {
+          xl[half * 128 + row] = l;
+          mbar_arrive(bar_ep);
+          wok = __all_sync(0xffffffffu, mbar_wait(bar_ep, 0, lim, abort_flag));
+          L = l + xl[(half ^ 1) * 128 + row];
+        }
       }
       if (!wok) {
         fail();
@@ -528,40 +593,44 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const bool empty = !(L > 0.0f);
         const float inv = empty ? 0.0f : vscale / L;
-        if (!empty) {
-          const float ref = DT == 0 ? yref : (float)eref;
-          lse_v = (ref + __log2f(L)) * 0.6931471805599453f;
-        }
-        __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) + (((int64_t)b * p.Sq + i) * p.Hq + h) * DV;
+        __nv_bfloat16* orow =
+            static_cast<__nv_bfloat16*>(p.out) + (((int64_t)b * p.Sq + i) * p.Hq + h) * DV + col_h;
 #pragma unroll 1
-        for (int ch = 0; ch < DV / 32; ++ch) {
+        for (int ch = 0; ch < 2; ++ch) {
           uint32_t o[32];
           if (n_kv > 0) {
-            tmem_ld32(tbase + lane_off + kColO + ch * 32, o);
+            tmem_ld32(tbase + lane_off + kColO + col_h + ch * 32, o);
             tmem_ld_wait();
           } else {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = 0u;
+            for (int q = 0; q < 32; ++q) o[q] = 0u;
           }
           uint32_t pk[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            pk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
+          for (int q = 0; q < 16; ++q)
+            pk[q] = pack_bf16x2(__uint_as_float(o[2 * q]) * inv, __uint_as_float(o[2 * q + 1]) * inv);
           if (i < p.Sq) {
             uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-              dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+            for (int q = 0; q < 4; ++q)
+              dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
           }
         }
-        if (p.lse && i < p.Sq) p.lse[((int64_t)b * p.Hq + h) * p.Sq + i] = lse_v;
+        if (half == 0 && p.lse && i < p.Sq) {
+          float lse_v = -INFINITY;
+          if (!empty) {
+            const float ref = DT == 0 ? yref : (float)eref;
+            lse_v = (ref + __log2f(L)) * 0.6931471805599453f;
+          }
+          p.lse[((int64_t)b * p.Hq + h) * p.Sq + i] = lse_v;
+        }
       }
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kWarpMma) {
     tc_fence_after();
     tmem_dealloc(tbase, kTmemCols);
   }

@@ -159,8 +159,9 @@ size_t zq_quantize_workspace_bytes(void) { return 256; }
 
 int zq_quantize_fp8(const void* x, int x_dtype, int64_t n_vec, int d, int hadamard,
                     void* x_fp8, float* descale, void* workspace, void* stream) {
-  if (!x || !x_fp8 || !descale || !workspace) return ZQ_ERR_NULL;
+  if (!descale || !workspace) return ZQ_ERR_NULL;
   if (n_vec < 0 || d <= 0) return ZQ_ERR_SHAPE;
+  if (n_vec > 0 && (!x || !x_fp8)) return ZQ_ERR_NULL;
   if (x_dtype != ZQ_X_F32 && x_dtype != ZQ_X_BF16) return ZQ_ERR_UNSUPPORTED;
   if (d % 8 != 0 || (hadamard && d % 128 != 0)) return ZQ_ERR_UNSUPPORTED;
   if (n_vec > (int64_t)1 << 40 || n_vec * (int64_t)d > ((int64_t)1 << 40)) return ZQ_ERR_SHAPE;

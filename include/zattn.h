@@ -133,9 +133,10 @@ ZQ_API int zq_attn_fwd_ex(const zq_attn_args* args, void* stream);
  * P words written for it, to the device buffer `dbg` (caller-owned,
  * ZQ_DEBUG_BYTES bytes): float S[128][128] (raw q.k dot products, no
  * scale), uint32 P[128][64] (bf16: 64 words of 2 x bf16; FP8: the first 32
- * words hold 4 x e4m3 each, key order little-endian), uint32 SF[128] (FP8:
- * UE8M0 scale bytes of the four 32-key chunks of each row).  For tests. */
-#define ZQ_DEBUG_BYTES (128 * 128 * 4 + 128 * 64 * 4 + 128 * 4)
+ * words hold 4 x e4m3 each, key order little-endian), uint32 SF[2][128]
+ * (FP8: the UE8M0 scale of 64-key block 0 / 1 of each row, repeated in all
+ * four bytes).  For tests. */
+#define ZQ_DEBUG_BYTES (128 * 128 * 4 + 128 * 64 * 4 + 256 * 4)
 ZQ_API int zq_attn_fwd_debug(const zq_attn_args* args, void* dbg, void* stream);
 
 /*
@@ -155,6 +156,7 @@ ZQ_API int zq_attn_fwd_debug(const zq_attn_args* args, void* dbg, void* stream);
  *   workspace  device scratch of zq_quantize_workspace_bytes() bytes, 16-byte
  *            aligned; its contents on entry do not matter and it must not be
  *            used by another call that runs at the same time.
+ * n_vec == 0 writes only the descale (0); x and x_fp8 may then be NULL.
  * Errors: ZQ_ERR_NULL, ZQ_ERR_SHAPE (n_vec < 0, d <= 0), ZQ_ERR_UNSUPPORTED
  *   (x_dtype, hadamard with d % 128 != 0, d % 8 != 0), ZQ_ERR_ALIGN (x,
  *   x_fp8, workspace not 16-byte aligned), ZQ_ERR_ARCH, ZQ_ERR_CUDA.

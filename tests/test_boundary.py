@@ -81,6 +81,7 @@ def test_attn_plain_entry_validates_too():
 @pytest.mark.parametrize("args,code", [
     ((None, 0, 4, 128, 0, A, A, A), zq.ZQ_ERR_NULL),
     ((A, 0, 4, 128, 0, None, A, A), zq.ZQ_ERR_NULL),
+    ((None, 0, 0, 128, 0, None, None, A), zq.ZQ_ERR_NULL),
     ((A, 0, 4, 128, 0, A, None, A), zq.ZQ_ERR_NULL),
     ((A, 0, 4, 128, 0, A, A, None), zq.ZQ_ERR_NULL),
     ((A, 0, -1, 128, 0, A, A, A), zq.ZQ_ERR_SHAPE),
