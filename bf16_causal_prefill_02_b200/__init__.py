@@ -18,7 +18,8 @@ import os
 import re
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libzattn.so")
+# ZQ_LIB_PATH selects another build of the same library (for comparing builds).
+LIB_PATH = os.environ.get("ZQ_LIB_PATH") or os.path.join(HERE, "libzattn.so")
 HEADER_PATH = os.path.join(os.path.dirname(HERE), "include", "zattn.h")
 
 ZQ_DTYPE_BF16, ZQ_DTYPE_FP8_E4M3 = 0, 1
@@ -60,7 +61,7 @@ def _load():
     lib.zq_attn_fwd.restype = i32
     lib.zq_attn_fwd_ex.argtypes = [ctypes.POINTER(zq_attn_args), P]
     lib.zq_attn_fwd_ex.restype = i32
-    lib.zq_attn_fwd_debug.argtypes = [ctypes.POINTER(zq_attn_args), P, P]
+    lib.zq_attn_fwd_debug.argtypes = [ctypes.POINTER(zq_attn_args), P, i32, i32, P]
     lib.zq_attn_fwd_debug.restype = i32
     lib.zq_quantize_fp8.argtypes = [P, i32, i64, i32, i32, P, P, P, P]
     lib.zq_quantize_fp8.restype = i32
@@ -94,11 +95,11 @@ def zq_attn_fwd_ex(args: zq_attn_args, stream) -> int:
     return _lib.zq_attn_fwd_ex(ctypes.byref(args), stream)
 
 
-def zq_attn_fwd_debug(args: zq_attn_args, dbg, stream) -> int:
-    return _lib.zq_attn_fwd_debug(ctypes.byref(args), dbg, stream)
+def zq_attn_fwd_debug(args: zq_attn_args, dbg, dbg_bh, dbg_qtile, stream) -> int:
+    return _lib.zq_attn_fwd_debug(ctypes.byref(args), dbg, dbg_bh, dbg_qtile, stream)
 
 
-ZQ_DEBUG_BYTES = 128 * 128 * 4 + 128 * 64 * 4 + 256 * 4
+ZQ_DEBUG_BYTES = 128 * 128 * 4 + 128 * 64 * 4 + 256 * 4 + 512 * 12 * 8
 
 
 def zq_quantize_fp8(x, x_dtype, n_vec, d, hadamard, x_fp8, descale, workspace, stream) -> int:
@@ -172,7 +173,7 @@ def quantize_fp8(x, hadamard: bool = False, out=None, descale=None, workspace=No
 
 def attn_fwd(q, k, v, out=None, lse=None, softmax_scale=None, causal=True, q_descale=None,
              k_descale=None, v_descale=None, softmax_mode=ZQ_SOFTMAX_LEANP, block_scale=True,
-             headroom_T=8, status=None, return_lse=True, stream=None, debug=None):
+             headroom_T=8, status=None, return_lse=True, stream=None, debug=None, debug_at=(0, 0)):
     """Causal prefill attention on CUDA tensors.
 
     q (B,Sq,Hq,d_qk), k (B,Sk,Hkv,d_qk), v (B,Sk,Hkv,d_v): bfloat16, or FP8
@@ -206,7 +207,8 @@ def attn_fwd(q, k, v, out=None, lse=None, softmax_scale=None, causal=True, q_des
     a.headroom_T = int(headroom_T)
     a.status = _ptr(status)
     if debug is not None:
-        _check(zq_attn_fwd_debug(a, debug.data_ptr(), _stream(stream)), "zq_attn_fwd_debug")
+        _check(zq_attn_fwd_debug(a, debug.data_ptr(), int(debug_at[0]), int(debug_at[1]), _stream(stream)),
+               "zq_attn_fwd_debug")
     else:
         _check(zq_attn_fwd_ex(a, _stream(stream)), "zq_attn_fwd_ex")
     return out, lse

@@ -16,19 +16,17 @@
 //        "How ZYFA works" (scaling by powers of 2 before rounding).
 //
 // One CTA computes one 128-row query tile of one (batch, head).  Warp roles:
-//   warps 0-7  softmax + epilogue.  Warps w and w+4 share TMEM lane quarter
-//              w%4, so thread t (t < 256) owns query row t%128 and the half
-//              h = t/128 of every 128-key tile: keys [64h, 64h+64), which is
-//              exactly one 64-key scaling block.
-//   warp 8     TMA producer (Q once, then K/V tiles through an NS-stage ring)
-//   warp 9     TMEM allocator and single-thread tcgen05.mma issuer
+//   warps 0-3  softmax + epilogue; thread t owns query row t (TMEM lane t)
+//   warp 4     TMA producer (Q once, then K/V tiles through an NS-stage ring)
+//   warp 5     TMEM allocator and single-thread tcgen05.mma issuer
 // Tensor memory (512 columns x 128 lanes, fp32 words):
 //   S0 [0,128) S1 [128,256)   score tiles; P (bf16x2 or 4 x e4m3 per word)
 //                             is written over the first columns of its S
 //   O  [256,256+DV)           output accumulator
 //   RS [384,400)              FP8: rounded row sum (P times a ones matrix)
-//   SFA [400,416)             FP8: UE8M0 scales of P, [buffer][half] x 4 cols
-//   SFB [416,420)             FP8: scales of V / ones, all 2^0
+//   SFA [400,408)             FP8: UE8M0 scales of P, one 4-column set per S
+//                             buffer (replicated layout, see sf_smem below)
+//   SFB [408,412)             FP8: scales of V / ones, all 2^0
 // MMA issue order: QK_0, QK_1, PV_0, QK_2, PV_1, ... so the softmax of tile
 // j+1 overlaps PV_j and QK_{j+2}.
 #include <cuda_fp8.h>
@@ -43,10 +41,10 @@
 namespace zq {
 
 constexpr int kTile = 128;
-constexpr int kSoftmaxThreads = 256;
+constexpr int kSoftmaxThreads = 128;
 constexpr int kThreads = kSoftmaxThreads + 64;
-constexpr int kWarpProducer = 8, kWarpMma = 9;
-constexpr uint32_t kColS0 = 0, kColO = 256, kColRS = 384, kColSFA = 400, kColSFB = 416;
+constexpr int kWarpProducer = 4, kWarpMma = 5;
+constexpr uint32_t kColS0 = 0, kColO = 256, kColRS = 384, kColSFA = 400, kColSFB = 408;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kInvalidExp = -(1 << 20);
 
@@ -67,11 +65,9 @@ struct Geo {
   static constexpr int OFF_K = OFF_Q + QBYTES;
   static constexpr int OFF_V = OFF_K + NS * KBYTES;
   static constexpr int OFF_ONES = OFF_V + NS * VBYTES;     // 16 x 128 keys e4m3, K-major
-  static constexpr int OFF_X = OFF_ONES + 2048;            // exchange: [2 buf][2 half][128] int
-  static constexpr int OFF_XR = OFF_X + 2048;              // [2 buf][128] int (reference)
-  static constexpr int OFF_XL = OFF_XR + 1024;             // [2 half][128] float (row sums)
-  static constexpr int OFF_BAR = OFF_XL + 1024;
-  static constexpr int NBAR = 1 + 4 * NS + 2 + 2 + 1 + 1 + 2 + 1;
+  static constexpr int OFF_SF = OFF_ONES + 2048;           // [2 buf][128] scale words
+  static constexpr int OFF_BAR = OFF_SF + 1024;
+  static constexpr int NBAR = 1 + 2 * NS + 2 + 2 + 2 + 1;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;  // + alignment slack
   static_assert(QBYTES % 1024 == 0 && VBYTES % 1024 == 0, "1 KB aligned tiles");
 };
@@ -117,10 +113,12 @@ __device__ __forceinline__ float pow2i(int e) {  // exact 2^e for -126 <= e <= 1
   return __int_as_float((e + 127) << 23);
 }
 // Max of 64 floats with four independent 3-input max chains.
+// (Lean P and the exact mode take one power-of-2 exponent per 64-key block.)
 __device__ __forceinline__ float max64(const float* s) {
-  float m0 = s[0], m1 = s[1], m2 = s[2], m3 = s[3];
+  float m0 = fmaxf(s[0], s[1]), m1 = fmaxf(s[2], s[3]);
+  float m2 = fmaxf(s[4], s[5]), m3 = fmaxf(s[6], s[7]);
 #pragma unroll
-  for (int c = 4; c < 64; c += 8) {
+  for (int c = 8; c < 64; c += 8) {
     m0 = max3(m0, s[c], s[c + 1]);
     m1 = max3(m1, s[c + 2], s[c + 3]);
     m2 = max3(m2, s[c + 4], s[c + 5]);
@@ -128,12 +126,31 @@ __device__ __forceinline__ float max64(const float* s) {
   }
   return fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
 }
-// Reference-exponent rule shared by both halves of a row (FP8): returns the
-// exponent E after seeing this tile's largest block exponent `emax`.
+// Reference-exponent rule (FP8): the row's exponent E after seeing this
+// tile's largest block exponent `emax`; it only moves up, and only when a
+// block exceeds it by more than `thr`.
 __device__ __forceinline__ int next_ref(int eref_old, int emax, int thr) {
   if (emax <= kInvalidExp) return eref_old;
   if (eref_old <= kInvalidExp) return emax;
   return emax > eref_old + thr ? emax : eref_old;
+}
+
+
+// Debug trace (clock64 of the traced CTA), per key tile j, 12 slots:
+//   [0] row 0 saw S_j  [1] row 0 loaded S_j  [2] row 0 computed P_j
+//   [3] row 0 released P_j  [4] row 96 released P_j
+//   MMA thread: [5] K_j landed, QK_j issue starts  [6] QK_j issued+committed
+//   [7] P_j seen  [8] V_j landed, PV_j issue starts  [9] PV_j MMAs issued
+//   [10] PV_j committed
+// Lives after the S/P/SF dump in the debug buffer.
+constexpr int kTraceOffsetWords = 128 * 128 + 128 * 64 + 256;
+constexpr int kTraceTiles = 512;
+constexpr int kTraceSlots = 12;
+
+__device__ __forceinline__ uint64_t clk64() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%clock64;" : "=l"(t));
+  return t;
 }
 
 template <int DT, int DQK, int DV, int MODE, int BS>
@@ -147,25 +164,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + G::OFF_BAR);
   uint64_t* bar_q = bars;
-  uint64_t* bar_kfull = bars + 1;
-  uint64_t* bar_kempty = bar_kfull + G::NS;
-  uint64_t* bar_vfull = bar_kempty + G::NS;
-  uint64_t* bar_vempty = bar_vfull + G::NS;
-  uint64_t* bar_sfull = bar_vempty + G::NS;  // [2]
-  uint64_t* bar_pfull = bar_sfull + 2;       // [2]
-  // bar_pvdone completes once per PV_j.  When softmax j (j >= 1) needs O it
-  // waits for phase j-1: PV_0..PV_{j-2} are complete (S_j's commit came
-  // after them) and PV_j cannot start before P_j, so exactly phases j-1 and
-  // j are possible and the parity test is unambiguous.
-  uint64_t* bar_pvdone = bar_pfull + 2;      // [1]
-  uint64_t* bar_ofinal = bar_pvdone + 1;     // [1] last PV landed
-  uint64_t* bar_x = bar_ofinal + 1;          // [2] per-tile exchange between halves
-  uint64_t* bar_ep = bar_x + 2;              // [1] epilogue exchange
+  uint64_t* bar_kvfull = bars + 1;           // [NS] K_j and V_j landed
+  // bar_kvdone[s] completes when PV_j (j = s mod NS) is done: it frees the
+  // K/V stage and tells the softmax that O holds tiles <= j.  Softmax j
+  // (j >= 1) waits for PV_{j-1}: of that stage's phases only (j-1)/NS - 1
+  // (done long ago) or (j-1)/NS can be complete, since PV_{j-1+NS} needs
+  // P_{j-1+NS}; so the parity test is unambiguous.
+  uint64_t* bar_kvdone = bar_kvfull + G::NS;  // [NS]
+  uint64_t* bar_sfull = bar_kvdone + G::NS;   // [2]
+  uint64_t* bar_pfull = bar_sfull + 2;        // [2]
+  uint64_t* bar_sf = bar_pfull + 2;           // [2] FP8: scale words staged
+  uint64_t* bar_ofinal = bar_sf + 2;          // [1] last PV landed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + G::NBAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int* xch = reinterpret_cast<int*>(smem + G::OFF_X);      // [2][2][128]
-  int* xref = reinterpret_cast<int*>(smem + G::OFF_XR);    // [2][128]
-  float* xl = reinterpret_cast<float*>(smem + G::OFF_XL);  // [2][128]
+  // FP8 scale words [buf][row], transposed through shared memory into the
+  // replicated TMEM layout the block-scaled MMA reads: query row r's word
+  // (byte k scales keys 32k..32k+31 of the tile) sits in TMEM column r/32 of
+  // the buffer's 4-column set, at lanes r%32 + 32q of every lane quarter q.
+  uint32_t* sf_smem = reinterpret_cast<uint32_t*>(smem + G::OFF_SF);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -182,23 +198,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int max_key = p.causal ? min(q1 + shift, p.Sk - 1) : p.Sk - 1;
   const int n_kv = max_key < 0 ? 0 : max_key / kTile + 1;
   const int min_lim = p.causal ? min(q0 + shift, p.Sk - 1) : p.Sk - 1;
+  const bool traced = p.dbg != nullptr && t == p.dbg_t && bh == p.dbg_bh;
+  uint64_t* trace = traced ? reinterpret_cast<uint64_t*>(static_cast<uint32_t*>(p.dbg) + kTraceOffsetWords)
+                           : nullptr;
 
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 1);
     for (int s = 0; s < G::NS; ++s) {
-      mbar_init(bar_kfull + s, 1);
-      mbar_init(bar_kempty + s, 1);
-      mbar_init(bar_vfull + s, 1);
-      mbar_init(bar_vempty + s, 1);
+      mbar_init(bar_kvfull + s, 1);
+      mbar_init(bar_kvdone + s, 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar_sfull + s, 1);
       mbar_init(bar_pfull + s, kSoftmaxThreads);
-      mbar_init(bar_x + s, kSoftmaxThreads);
+      mbar_init(bar_sf + s, kSoftmaxThreads);
     }
-    mbar_init(bar_pvdone, 1);
     mbar_init(bar_ofinal, 1);
-    mbar_init(bar_ep, kSoftmaxThreads);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -244,85 +259,93 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       for (int j = 0; j < n_kv; ++j) {
         const int s = j % G::NS;
-        const uint32_t ph = ((j / G::NS) & 1) ^ 1;
-        if (!mbar_wait(bar_kempty + s, ph, lim, abort_flag)) { fail(); break; }
+        const uint32_t ph = ((j / G::NS) & 1) ^ 1;  // first pass through the ring: free
+        if (!mbar_wait(bar_kvdone + s, ph, lim, abort_flag)) { fail(); break; }
         uint8_t* sk = smem + G::OFF_K + s * G::KBYTES;
-        mbar_arrive_expect_tx(bar_kfull + s, G::KBYTES);
+        uint8_t* sv = smem + G::OFF_V + s * G::VBYTES;
+        mbar_arrive_expect_tx(bar_kvfull + s, G::KBYTES + G::VBYTES);
 #pragma unroll
         for (int c = 0; c < G::NCH; ++c) {
           const bool narrow = (c == G::NCH - 1) && G::LASTW == 64;
           tma_load_4d(sk + c * 16384, narrow ? (const void*)&tmK2 : (const void*)&tmK,
-                      bar_kfull + s, c * 128 / G::ES, g, j * kTile, b);
+                      bar_kvfull + s, c * 128 / G::ES, g, j * kTile, b);
         }
-        if (!mbar_wait(bar_vempty + s, ph, lim, abort_flag)) { fail(); break; }
-        uint8_t* sv = smem + G::OFF_V + s * G::VBYTES;
-        mbar_arrive_expect_tx(bar_vfull + s, G::VBYTES);
 #pragma unroll
         for (int c = 0; c < G::VCH; ++c)
-          tma_load_4d(sv + c * 16384, &tmV, bar_vfull + s, c * 128 / G::ES, g, j * kTile, b);
+          tma_load_4d(sv + c * 16384, &tmV, bar_kvfull + s, c * 128 / G::ES, g, j * kTile, b);
       }
     }
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
+    // One thread; tcgen05.mma issue runs nearly in step with execution, so
+    // this loop is on the critical path: descriptors are built once, each
+    // tile costs one K/V wait, one P wait and two commits.
     if (lane == 0 && n_kv > 0) {
       const uint32_t sbase = smem_u32(smem);
       constexpr uint32_t idesc_qk = idesc_dense(DT == 0 ? 1u : 0u, 0u, 128, 128);
       constexpr uint32_t idesc_pv_bf16 = idesc_dense(1u, 1u, 128, DV);
-      auto qk_desc = [&](uint32_t base, int kk) -> uint64_t {
+      // descriptors of stage 0; stage s adds its byte offset >> 4 to the
+      // 14-bit start-address field (all addresses stay below 256 KB)
+      uint64_t dq[G::QK_STEPS], dk[G::QK_STEPS], dvv[G::PV_STEPS], d1[4];
+#pragma unroll
+      for (int kk = 0; kk < G::QK_STEPS; ++kk) {
         const int pos = kk * 32;
         const int c = pos / 128;
         const bool narrow = (c == G::NCH - 1) && G::LASTW == 64;
-        return smem_desc(base + c * 16384 + (pos % 128), 16, narrow ? 512 : 1024,
-                         narrow ? SW_64B : SW_128B);
-      };
+        const uint32_t off = c * 16384 + (pos % 128);
+        dq[kk] = smem_desc(sbase + G::OFF_Q + off, 16, narrow ? 512 : 1024, narrow ? SW_64B : SW_128B);
+        dk[kk] = smem_desc(sbase + G::OFF_K + off, 16, narrow ? 512 : 1024, narrow ? SW_64B : SW_128B);
+      }
+#pragma unroll
+      for (int kk = 0; kk < G::PV_STEPS; ++kk)  // 16 (bf16) or 32 (fp8) keys of V per step
+        dvv[kk] = smem_desc(sbase + G::OFF_V + kk * (DT == 0 ? 16 : 32) * 128, 16384, 1024, SW_128B);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        d1[kk] = smem_desc(sbase + G::OFF_ONES + kk * 32, 16, 1024, SW_128B);
       auto issue_qk = [&](int j) -> bool {
         const int s = j % G::NS;
-        if (!mbar_wait(bar_kfull + s, (j / G::NS) & 1, lim, abort_flag)) return false;
+        if (!mbar_wait(bar_kvfull + s, (j / G::NS) & 1, lim, abort_flag)) return false;
         tc_fence_after();
+        if (trace && j < kTraceTiles) trace[j * kTraceSlots + 5] = clk64();
         const uint32_t dS = tbase + kColS0 + (j & 1) * 128;
-        const uint32_t kb = sbase + G::OFF_K + s * G::KBYTES;
-        const uint32_t qb = sbase + G::OFF_Q;
+        const uint64_t koff = (uint64_t)((s * G::KBYTES) >> 4);
 #pragma unroll
         for (int kk = 0; kk < G::QK_STEPS; ++kk) {
           if (DT == 0)
-            mma_f16_ss(dS, qk_desc(qb, kk), qk_desc(kb, kk), idesc_qk, kk > 0);
+            mma_f16_ss(dS, dq[kk], dk[kk] + koff, idesc_qk, kk > 0);
           else
-            mma_f8_ss(dS, qk_desc(qb, kk), qk_desc(kb, kk), idesc_qk, kk > 0);
+            mma_f8_ss(dS, dq[kk], dk[kk] + koff, idesc_qk, kk > 0);
         }
-        tc_commit(bar_kempty + s);
         tc_commit(bar_sfull + (j & 1));
+        if (trace && j < kTraceTiles) trace[j * kTraceSlots + 6] = clk64();
         return true;
       };
       auto issue_pv = [&](int j) -> bool {
         const int s = j % G::NS;
         if (!mbar_wait(bar_pfull + (j & 1), (j >> 1) & 1, lim, abort_flag)) return false;
-        if (!mbar_wait(bar_vfull + s, (j / G::NS) & 1, lim, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t vb = sbase + G::OFF_V + s * G::VBYTES;
+        if (trace && j < kTraceTiles) trace[j * kTraceSlots + 8] = clk64();
+        const uint64_t voff = (uint64_t)((s * G::VBYTES) >> 4);
         const uint32_t aP = tbase + kColS0 + (j & 1) * 128;
 #pragma unroll
         for (int kk = 0; kk < G::PV_STEPS; ++kk) {
           const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
           if (DT == 0) {
-            // 16 keys per step = 8 packed bf16x2 columns of P; V rows 16*kk..
-            const uint64_t dv = smem_desc(vb + kk * 16 * 128, 16384, 1024, SW_128B);
-            mma_f16_ts(tbase + kColO, aP + kk * 8, dv, idesc_pv_bf16, acc);
+            // 16 keys per step = 8 packed bf16x2 columns of P
+            mma_f16_ts(tbase + kColO, aP + kk * 8, dvv[kk] + voff, idesc_pv_bf16, acc);
           } else {
-            // 32 keys per step = 8 columns of 4 x e4m3.  Keys 32kk.. belong to
-            // half kk/2; its scale word sits in SFA[buf][kk/2], byte kk%2.
-            const uint64_t dv = smem_desc(vb + kk * 32 * 128, 16384, 1024, SW_128B);
-            const uint32_t sid = (uint32_t)(kk & 1);
-            const uint32_t sfa = (tbase + kColSFA + (j & 1) * 8 + (kk >> 1) * 4) | (sid << 30);
-            const uint32_t sfb = (tbase + kColSFB) | (sid << 30);
-            mma_mxf8_ts(tbase + kColO, aP + kk * 8, dv, idesc_mx(1u, 128, DV, sid, sid), sfa, sfb,
+            // 32 keys per step = 8 columns of 4 x e4m3; scale byte kk
+            const uint32_t sfa = (tbase + kColSFA + (j & 1) * 4) | ((uint32_t)kk << 30);
+            const uint32_t sfb = (tbase + kColSFB) | ((uint32_t)kk << 30);
+            mma_mxf8_ts(tbase + kColO, aP + kk * 8, dvv[kk] + voff, idesc_mx(1u, 128, DV, kk, kk),
+                        sfa, sfb, acc);
+            mma_mxf8_ts(tbase + kColRS, aP + kk * 8, d1[kk], idesc_mx(0u, 128, 16, kk, kk), sfa, sfb,
                         acc);
-            const uint64_t d1 = smem_desc(sbase + G::OFF_ONES + kk * 32, 16, 1024, SW_128B);
-            mma_mxf8_ts(tbase + kColRS, aP + kk * 8, d1, idesc_mx(0u, 128, 16, sid, sid), sfa,
-                        sfb, acc);
           }
         }
-        tc_commit(bar_vempty + s);
-        tc_commit(bar_pvdone);
+        if (trace && j < kTraceTiles) trace[j * kTraceSlots + 9] = clk64();
+        tc_commit(bar_kvdone + s);
+        if (trace && j < kTraceTiles) trace[j * kTraceSlots + 10] = clk64();
         return true;
       };
       bool ok = true;
@@ -337,13 +360,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------ softmax (rows)
-    const int half = threadIdx.x >> 7;  // which 64-key block of each tile
-    const int row = threadIdx.x & 127;  // query row == TMEM lane
-    const int quarter = warp & 3;
+    const int row = threadIdx.x;  // query row == TMEM lane
     const int i = q0 + row;
     const int row_lim = p.causal ? min(i + shift, p.Sk - 1) : p.Sk - 1;
-    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    const uint32_t col_h = (uint32_t)half * 64;  // first S / O column of this half
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     float c = p.softmax_scale * 1.4426950408889634f;  // log2(e)
     float vscale = 1.0f;
     if (DT == 1) {
@@ -351,22 +371,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float kd = p.k_descale ? *p.k_descale : 1.0f;
       vscale = p.v_descale ? *p.v_descale : 1.0f;
       c = ((p.softmax_scale * qd) * kd) * 1.4426950408889634f;
-      if (half == 0) {
-        // SFB (scales of V and of the ones matrix): all 2^0 = 0x7F
-        tmem_st4(tbase + lane_off + kColSFB, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
-      } else if (!BS) {
-        // running mode: every block scale is 2^0 as well
+      // SFB (scales of V and of the ones matrix): all 2^0 = 0x7F
+      tmem_st4(tbase + lane_off + kColSFB, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+      if (!BS) {  // running mode: every block scale is 2^0 as well
         tmem_st4(tbase + lane_off + kColSFA, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
         tmem_st4(tbase + lane_off + kColSFA + 4, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
-        tmem_st4(tbase + lane_off + kColSFA + 8, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
-        tmem_st4(tbase + lane_off + kColSFA + 12, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
       }
       tmem_st_wait();
     }
     const int T = p.headroom_T;
     float yref = -INFINITY;   // BF16 / FP8 running mode: log2-domain reference
     int eref = kInvalidExp;   // FP8: reference exponent E (invalid until a key is seen)
-    float l = 0.0f;           // BF16 partial row sum over this half (fp32, unrounded p)
+    float l = 0.0f;           // BF16 row sum (fp32, unrounded p)
     bool ok = true;
 
     for (int j = 0; ok && j < n_kv; ++j) {
@@ -374,41 +390,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool w = mbar_wait(bar_sfull + buf, (j >> 1) & 1, lim, abort_flag);
       if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
       tc_fence_after();
-      uint32_t sr[64];
+      if (trace && row == 0 && j < kTraceTiles) trace[j * kTraceSlots + 0] = clk64();
+      float s[128];  // explicit bit casts: no type punning through pointers
       {
-        uint32_t(&a0)[32] = *reinterpret_cast<uint32_t(*)[32]>(sr);
-        uint32_t(&a1)[32] = *reinterpret_cast<uint32_t(*)[32]>(sr + 32);
-        const uint32_t ts = tbase + lane_off + kColS0 + buf * 128 + col_h;
+        uint32_t a0[32], a1[32], a2[32], a3[32];
+        const uint32_t ts = tbase + lane_off + kColS0 + buf * 128;
         tmem_ld32(ts, a0);
         tmem_ld32(ts + 32, a1);
+        tmem_ld32(ts + 64, a2);
+        tmem_ld32(ts + 96, a3);
         tmem_ld_wait();
+#pragma unroll
+        for (int cc = 0; cc < 32; ++cc) {
+          s[cc] = __uint_as_float(a0[cc]);
+          s[32 + cc] = __uint_as_float(a1[cc]);
+          s[64 + cc] = __uint_as_float(a2[cc]);
+          s[96 + cc] = __uint_as_float(a3[cc]);
+        }
       }
-      float* s = reinterpret_cast<float*>(sr);
-      const bool dump = p.dbg != nullptr && j == 0 && t == 0 && bh == 0;
+      if (trace && row == 0 && j < kTraceTiles) trace[j * kTraceSlots + 1] = clk64();
+      const bool dump = traced && j == 0;
       if (dump) {
-        float* ds = static_cast<float*>(p.dbg) + row * 128 + col_h;
+        float* ds = static_cast<float*>(p.dbg) + row * 128;
 #pragma unroll
-        for (int cc = 0; cc < 64; ++cc) ds[cc] = s[cc];
+        for (int cc = 0; cc < 128; ++cc) ds[cc] = s[cc];
       }
-      const int kbase = j * kTile + (int)col_h;
-      if (kbase + 63 > min_lim) {
+      const int kbase = j * kTile;
+      if (kbase + kTile - 1 > min_lim) {
 #pragma unroll
-        for (int cc = 0; cc < 64; ++cc)
+        for (int cc = 0; cc < 128; ++cc)
           if (kbase + cc > row_lim) s[cc] = -INFINITY;
       }
-      const float m = max64(s);  // raw block maximum (scores before scaling)
-      int* xb = xch + buf * 256;
-      int* xr = xref + buf * 128;
+      const float m0 = max64(s), m1 = max64(s + 64);  // raw block maxima
+      const uint32_t tP = tbase + lane_off + kColS0 + buf * 128;
 
       if constexpr (DT == 0) {
         // ------------------------------------------------ BF16, exact exp2
-        xb[half * 128 + row] = __float_as_int(m);
-        tc_fence_before();  // both halves' S loads complete before any P store
-        mbar_arrive(bar_x + buf);
-        w = mbar_wait(bar_x + buf, (j >> 1) & 1, lim, abort_flag);
-        if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
-        tc_fence_after();
-        const float ymax = fmaxf(m, __int_as_float(xb[(half ^ 1) * 128 + row])) * c;
+        const float ymax = fmaxf(m0, m1) * c;
         const bool need = ymax > yref + 8.0f;
         if (__any_sync(0xffffffffu, need)) {
           const float nref = fmaxf(yref, ymax);
@@ -417,26 +435,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           l *= f;
           if (j > 0) {
             // O holds tiles < j; PV_{j-1} must have landed before rescaling
-            w = mbar_wait(bar_pvdone, (j - 1) & 1, lim, abort_flag);
+            w = mbar_wait(bar_kvdone + (j - 1) % G::NS, ((j - 1) / G::NS) & 1, lim, abort_flag);
             if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
             tc_fence_after();
 #pragma unroll 1
-            for (int ch = 0; ch < 2; ++ch) {
+            for (int ch = 0; ch < DV / 32; ++ch) {
               uint32_t o[32];
-              const uint32_t to = tbase + lane_off + kColO + col_h + ch * 32;
+              const uint32_t to = tbase + lane_off + kColO + ch * 32;
               tmem_ld32(to, o);
               tmem_ld_wait();
 #pragma unroll
-              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+              for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * f);
               tmem_st32(to, o);
             }
           }
         }
         const float nb = yref == -INFINITY ? 0.0f : -yref;
-        uint32_t pk[32];
+        uint32_t pk[64];
         float lp0 = 0.0f, lp1 = 0.0f;
 #pragma unroll
-        for (int cc = 0; cc < 64; cc += 2) {
+        for (int cc = 0; cc < 128; cc += 2) {
           float z0, z1;
           ffma2(z0, z1, s[cc], s[cc + 1], c, nb);
           const float p0 = ex2_approx(z0);
@@ -446,141 +464,129 @@ __global__ void __launch_bounds__(kThreads, 1)
           pk[cc / 2] = pack_bf16x2(p0, p1);
         }
         l += lp0 + lp1;
-        tmem_st32(tbase + lane_off + kColS0 + buf * 128 + half * 32, pk);
+        if (trace && row == 0 && j < kTraceTiles) trace[j * kTraceSlots + 2] = clk64();
+        tmem_st32(tP, *reinterpret_cast<uint32_t(*)[32]>(pk));
+        tmem_st32(tP + 32, *reinterpret_cast<uint32_t(*)[32]>(pk + 32));
         if (dump) {
-          uint32_t* dp = reinterpret_cast<uint32_t*>(static_cast<float*>(p.dbg) + 128 * 128);
+          uint32_t* dp = static_cast<uint32_t*>(p.dbg) + 128 * 128;
 #pragma unroll
-          for (int e = 0; e < 32; ++e) dp[row * 64 + half * 32 + e] = pk[e];
+          for (int q = 0; q < 64; ++q) dp[row * 64 + q] = pk[q];
         }
       } else {
         // ------------------------------------------------ FP8 P path
-        int e;  // this half's block exponent
-        if (BS) {
-          e = m != -INFINITY ? (int)ceilf(m * c) - T : kInvalidExp;
-          xb[half * 128 + row] = e;
-          if (half == 0) xr[row] = eref;
-        } else {
-          xb[half * 128 + row] = __float_as_int(m);
-        }
-        tc_fence_before();  // both halves' S loads complete before any P store
-        mbar_arrive(bar_x + buf);
-        w = mbar_wait(bar_x + buf, (j >> 1) & 1, lim, abort_flag);
-        if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
-        tc_fence_after();
+        int e0, e1;  // block exponents of keys [0,64) and [64,128)
         int nref;
         if (BS) {
-          nref = next_ref(eref, max(e, xb[(half ^ 1) * 128 + row]), 32);
+          e0 = m0 != -INFINITY ? (int)ceilf(m0 * c) - T : kInvalidExp;
+          e1 = m1 != -INFINITY ? (int)ceilf(m1 * c) - T : kInvalidExp;
+          nref = next_ref(eref, max(e0, e1), 32);
         } else {
           // running mode: one exponent from the running max of the row
-          const float mm = fmaxf(m, __int_as_float(xb[(half ^ 1) * 128 + row]));
-          yref = fmaxf(mm * c, yref);
+          yref = fmaxf(fmaxf(m0, m1) * c, yref);
           nref = yref != -INFINITY ? (int)ceilf(yref) - T : kInvalidExp;
-          e = nref;
+          e0 = e1 = nref;
         }
-        const bool had = eref > kInvalidExp;
-        const bool grow = had && nref != eref;
+        const bool grow = eref > kInvalidExp && nref != eref;
         if (j > 0 && __any_sync(0xffffffffu, grow)) {
           // O and the row sum hold tiles < j at scale 2^(-eref): move them to
           // 2^(-nref) exactly.  PV_{j-1} must have landed first.
           const float f = grow ? pow2i(max(eref - nref, -126)) : 1.0f;
-          w = mbar_wait(bar_pvdone, (j - 1) & 1, lim, abort_flag);
+          w = mbar_wait(bar_kvdone + (j - 1) % G::NS, ((j - 1) / G::NS) & 1, lim, abort_flag);
           if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll 1
-          for (int ch = 0; ch < 2; ++ch) {
+          for (int ch = 0; ch < DV / 32; ++ch) {
             uint32_t o[32];
-            const uint32_t to = tbase + lane_off + kColO + col_h + ch * 32;
+            const uint32_t to = tbase + lane_off + kColO + ch * 32;
             tmem_ld32(to, o);
             tmem_ld_wait();
 #pragma unroll
             for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * f);
             tmem_st32(to, o);
           }
-          if (half == 0) {
-            uint32_t rs;
-            tmem_ld1(tbase + lane_off + kColRS, rs);
-            tmem_ld_wait();
-            tmem_st1(tbase + lane_off + kColRS, __float_as_uint(__uint_as_float(rs) * f));
-          }
+          uint32_t rs;
+          tmem_ld1(tbase + lane_off + kColRS, rs);
+          tmem_ld_wait();
+          tmem_st1(tbase + lane_off + kColRS, __float_as_uint(__uint_as_float(rs) * f));
         }
         eref = nref;
-        const bool valid = e > kInvalidExp;
-        uint32_t pk[16];
+        const bool v0 = e0 > kInvalidExp, v1 = e1 > kInvalidExp;
+        uint32_t pk[32];
         if (MODE == 0) {
           // exact: e4m3_rne(exp2(y - e))
-          const float ne = valid ? -(float)e : 0.0f;
 #pragma unroll
-          for (int cc = 0; cc < 64; cc += 4) {
-            float z0, z1, z2, z3;
-            ffma2(z0, z1, s[cc], s[cc + 1], c, ne);
-            ffma2(z2, z3, s[cc + 2], s[cc + 3], c, ne);
-            pk[cc / 4] = pack_e4m3x4(ex2_approx(z0), ex2_approx(z1), ex2_approx(z2), ex2_approx(z3));
+          for (int blk = 0; blk < 2; ++blk) {
+            const float ne = blk == 0 ? (v0 ? -(float)e0 : 0.0f) : (v1 ? -(float)e1 : 0.0f);
+#pragma unroll
+            for (int cc = blk * 64; cc < blk * 64 + 64; cc += 4) {
+              float z0, z1, z2, z3;
+              ffma2(z0, z1, s[cc], s[cc + 1], c, ne);
+              ffma2(z2, z3, s[cc + 2], s[cc + 3], c, ne);
+              pk[cc / 4] =
+                  pack_e4m3x4(ex2_approx(z0), ex2_approx(z1), ex2_approx(z2), ex2_approx(z3));
+            }
           }
         } else {
           // Lean P: u = sat((8(y - e) + 56) / 128) clamps the code at 0; the
           // magic add 1.5*2^23 rounds 128u half-to-even into the low byte.
-          const float a = c * 0.0625f;                         // 8c / 128
-          const float k0 = valid ? (float)(56 - 8 * e) * 0.0078125f : 0.0f;
+          const float a = c * 0.0625f;  // 8c / 128
           const float magic = 12582912.0f;
 #pragma unroll
-          for (int cc = 0; cc < 64; cc += 4) {
-            const float u0 = fma_sat(s[cc], a, k0);
-            const float u1 = fma_sat(s[cc + 1], a, k0);
-            const float u2 = fma_sat(s[cc + 2], a, k0);
-            const float u3 = fma_sat(s[cc + 3], a, k0);
-            float x0, x1, x2, x3;
-            ffma2(x0, x1, u0, u1, 128.0f, magic);
-            ffma2(x2, x3, u2, u3, 128.0f, magic);
-            pk[cc / 4] = prmt(prmt(__float_as_uint(x0), __float_as_uint(x1), 0x0040u),
-                              prmt(__float_as_uint(x2), __float_as_uint(x3), 0x0040u), 0x5410u);
+          for (int blk = 0; blk < 2; ++blk) {
+            const int e = blk == 0 ? e0 : e1;
+            const bool v = blk == 0 ? v0 : v1;
+            const float k0 = v ? (float)(56 - 8 * e) * 0.0078125f : 0.0f;
+#pragma unroll
+            for (int cc = blk * 64; cc < blk * 64 + 64; cc += 4) {
+              const float u0 = fma_sat(s[cc], a, k0);
+              const float u1 = fma_sat(s[cc + 1], a, k0);
+              const float u2 = fma_sat(s[cc + 2], a, k0);
+              const float u3 = fma_sat(s[cc + 3], a, k0);
+              float x0, x1, x2, x3;
+              ffma2(x0, x1, u0, u1, 128.0f, magic);
+              ffma2(x2, x3, u2, u3, 128.0f, magic);
+              pk[cc / 4] = prmt(prmt(__float_as_uint(x0), __float_as_uint(x1), 0x0040u),
+                                prmt(__float_as_uint(x2), __float_as_uint(x3), 0x0040u), 0x5410u);
+            }
           }
         }
-        tmem_st16(tbase + lane_off + kColS0 + buf * 128 + half * 16, pk);
+        if (trace && row == 0 && j < kTraceTiles) trace[j * kTraceSlots + 2] = clk64();
+        tmem_st32(tP, pk);
+        const int sf0 = v0 ? min(max(e0 - eref + 127, 0), 254) : 0;
+        const int sf1 = v1 ? min(max(e1 - eref + 127, 0), 254) : 0;
+        const uint32_t sfw = (uint32_t)sf0 * 0x0101u | ((uint32_t)sf1 * 0x0101u) << 16;
         if (BS) {
-          // scale words for the four rows this thread's lane serves in the
-          // replicated SFA layout: column r/32 holds row r at lanes r%32+32q
-          uint32_t sw[4];
-#pragma unroll
-          for (int m1 = 0; m1 < 4; ++m1) {
-            const int rr = lane + 32 * m1;
-            const int ea = xb[rr], eb = xb[128 + rr];
-            const int en = next_ref(xr[rr], max(ea, eb), 32);
-            const int eo = half == 0 ? ea : eb;
-            const int sf = eo > kInvalidExp ? min(max(eo - en + 127, 0), 254) : 0;
-            sw[m1] = (uint32_t)sf * 0x01010101u;
-          }
-          tmem_st4(tbase + lane_off + kColSFA + buf * 8 + half * 4, sw[0], sw[1], sw[2], sw[3]);
+          sf_smem[buf * 128 + row] = sfw;
+          mbar_arrive(bar_sf + buf);
+          w = mbar_wait(bar_sf + buf, (j >> 1) & 1, lim, abort_flag);
+          if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+          tmem_st4(tbase + lane_off + kColSFA + buf * 4, sf_smem[buf * 128 + lane],
+                   sf_smem[buf * 128 + 32 + lane], sf_smem[buf * 128 + 64 + lane],
+                   sf_smem[buf * 128 + 96 + lane]);
         }
         if (dump) {
-          uint32_t* dp = reinterpret_cast<uint32_t*>(static_cast<float*>(p.dbg) + 128 * 128);
+          uint32_t* dp = static_cast<uint32_t*>(p.dbg) + 128 * 128;
 #pragma unroll
-          for (int q = 0; q < 16; ++q) dp[row * 64 + half * 16 + q] = pk[q];
-          dp[128 * 64 + half * 128 + row] =
-              valid ? (uint32_t)min(max(e - eref + 127, 0), 254) * 0x01010101u : 0u;
+          for (int q = 0; q < 32; ++q) dp[row * 64 + q] = pk[q];
+          dp[128 * 64 + row] = (uint32_t)sf0 * 0x01010101u;
+          dp[128 * 64 + 128 + row] = (uint32_t)sf1 * 0x01010101u;
         }
       }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar_pfull + buf);
+      if (trace && j < kTraceTiles) {
+        if (row == 0) trace[j * kTraceSlots + 3] = clk64();
+        if (row == 96) trace[j * kTraceSlots + 4] = clk64();
+      }
     }
     if (!ok) {
       fail();
     } else {
       // ------------------------------------------------------------ epilogue
+      float L = l, lse_v = -INFINITY;
       bool wok = true;
-      if (n_kv > 0) {
-        wok = mbar_wait(bar_ofinal, 0, lim, abort_flag);
-        wok = __all_sync(0xffffffffu, wok);
-      }
-      float L = 0.0f;
-      if (wok) {
-        if (DT == 0) {
-          xl[half * 128 + row] = l;
-          mbar_arrive(bar_ep);
-          wok = __all_sync(0xffffffffu, mbar_wait(bar_ep, 0, lim, abort_flag));
-          L = l + xl[(half ^ 1) * 128 + row];
-        }
-      }
+      if (n_kv > 0) wok = __all_sync(0xffffffffu, mbar_wait(bar_ofinal, 0, lim, abort_flag));
       if (!wok) {
         fail();
       } else {
@@ -593,13 +599,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const bool empty = !(L > 0.0f);
         const float inv = empty ? 0.0f : vscale / L;
+        if (!empty) {
+          const float ref = DT == 0 ? yref : (float)eref;
+          lse_v = (ref + __log2f(L)) * 0.6931471805599453f;
+        }
         __nv_bfloat16* orow =
-            static_cast<__nv_bfloat16*>(p.out) + (((int64_t)b * p.Sq + i) * p.Hq + h) * DV + col_h;
+            static_cast<__nv_bfloat16*>(p.out) + (((int64_t)b * p.Sq + i) * p.Hq + h) * DV;
 #pragma unroll 1
-        for (int ch = 0; ch < 2; ++ch) {
+        for (int ch = 0; ch < DV / 32; ++ch) {
           uint32_t o[32];
           if (n_kv > 0) {
-            tmem_ld32(tbase + lane_off + kColO + col_h + ch * 32, o);
+            tmem_ld32(tbase + lane_off + kColO + ch * 32, o);
             tmem_ld_wait();
           } else {
 #pragma unroll
@@ -616,14 +626,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
           }
         }
-        if (half == 0 && p.lse && i < p.Sq) {
-          float lse_v = -INFINITY;
-          if (!empty) {
-            const float ref = DT == 0 ? yref : (float)eref;
-            lse_v = (ref + __log2f(L)) * 0.6931471805599453f;
-          }
-          p.lse[((int64_t)b * p.Hq + h) * p.Sq + i] = lse_v;
-        }
+        if (p.lse && i < p.Sq) p.lse[((int64_t)b * p.Hq + h) * p.Sq + i] = lse_v;
       }
     }
   }

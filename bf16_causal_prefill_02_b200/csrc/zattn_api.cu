@@ -7,7 +7,7 @@
 #include <cmath>
 #include <cstdint>
 
-#include "../../include/zattn.h"
+#include "zattn.h"
 
 #include "zq_internal.h"
 
@@ -82,7 +82,7 @@ const char* zq_status_string(int s) {
   }
 }
 
-static int attn_impl(const zq_attn_args* a, void* dbg, void* stream) {
+static int attn_impl(const zq_attn_args* a, void* dbg, int dbg_bh, int dbg_t, void* stream) {
   int rc = validate_attn(a);
   if (rc != ZQ_OK) return rc;
   rc = check_device(nullptr);
@@ -114,15 +114,17 @@ static int attn_impl(const zq_attn_args* a, void* dbg, void* stream) {
       a->softmax_scale > 0.0f ? a->softmax_scale : (float)(1.0 / std::sqrt((double)a->d_qk));
   L.p.timeout_ns = kTimeoutNs;
   L.p.dbg = dbg;
+  L.p.dbg_bh = dbg_bh;
+  L.p.dbg_t = dbg_t;
   cudaError_t e = zq::launch_attention(L, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? ZQ_OK : ZQ_ERR_CUDA;
 }
 
-int zq_attn_fwd_ex(const zq_attn_args* a, void* stream) { return attn_impl(a, nullptr, stream); }
+int zq_attn_fwd_ex(const zq_attn_args* a, void* stream) { return attn_impl(a, nullptr, 0, 0, stream); }
 
-int zq_attn_fwd_debug(const zq_attn_args* a, void* dbg, void* stream) {
+int zq_attn_fwd_debug(const zq_attn_args* a, void* dbg, int dbg_bh, int dbg_qtile, void* stream) {
   if (!dbg) return ZQ_ERR_NULL;
-  return attn_impl(a, dbg, stream);
+  return attn_impl(a, dbg, dbg_bh, dbg_qtile, stream);
 }
 
 int zq_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B,

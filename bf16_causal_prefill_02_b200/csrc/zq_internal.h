@@ -20,10 +20,11 @@ struct AttnParams {
   int headroom_T;
   float softmax_scale;
   uint64_t timeout_ns;
-  // Debug dump (nullptr in normal use): the CTA of (batch 0, head 0, query
-  // tile 0) writes its first score tile, P words and scale words here:
-  // float S[128][128]; uint32 P[128][64]; uint32 SF[128].
+  // Debug dump (nullptr in normal use): the CTA of flat (batch*Hq + head)
+  // dbg_bh and query tile dbg_t writes its first score tile, P words and
+  // scale words here: float S[128][128]; uint32 P[128][64]; uint32 SF[2][128].
   void* dbg;
+  int dbg_bh, dbg_t;
 };
 
 struct AttnLaunch {

@@ -128,16 +128,19 @@ typedef struct zq_attn_args {
  * range (they are ignored, not checked, for bf16). */
 ZQ_API int zq_attn_fwd_ex(const zq_attn_args* args, void* stream);
 
-/* zq_attn_fwd_debug -- zq_attn_fwd_ex that also dumps, for (batch 0,
- * head 0, query tile 0), the first 128x128 score tile before masking and the
+/* zq_attn_fwd_debug -- zq_attn_fwd_ex that also dumps, for the query tile
+ * dbg_qtile (rows 128*dbg_qtile..) of flat head dbg_bh = batch*Hq + head,
+ * the first 128x128 score tile before masking and the
  * P words written for it, to the device buffer `dbg` (caller-owned,
  * ZQ_DEBUG_BYTES bytes): float S[128][128] (raw q.k dot products, no
  * scale), uint32 P[128][64] (bf16: 64 words of 2 x bf16; FP8: the first 32
  * words hold 4 x e4m3 each, key order little-endian), uint32 SF[2][128]
  * (FP8: the UE8M0 scale of 64-key block 0 / 1 of each row, repeated in all
- * four bytes).  For tests. */
-#define ZQ_DEBUG_BYTES (128 * 128 * 4 + 128 * 64 * 4 + 256 * 4)
-ZQ_API int zq_attn_fwd_debug(const zq_attn_args* args, void* dbg, void* stream);
+ * four bytes), then uint64 TRACE[512][12]: SM clock (clock64) at twelve points of
+ * the pipeline for key tile j (see attn_fwd.cu).  For tests and tuning. */
+#define ZQ_DEBUG_BYTES (128 * 128 * 4 + 128 * 64 * 4 + 256 * 4 + 512 * 12 * 8)
+ZQ_API int zq_attn_fwd_debug(const zq_attn_args* args, void* dbg, int dbg_bh, int dbg_qtile,
+                             void* stream);
 
 /*
  * zq_quantize_fp8 -- per-tensor FP8 e4m3 quantiser with an optional fused

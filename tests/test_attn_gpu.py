@@ -70,6 +70,15 @@ def test_debug_exact_codes_match_emulation():
 
 
 @pytest.mark.parametrize("dtype", DTYPES)
+def test_row_with_single_very_negative_score(dtype):
+    # Row 0 sees one key whose score is far below every other row's scores;
+    # its block exponent must come from its own (masked) block.
+    q, k, v = workloads.make_custom(1, 256, 256, 2, 2, 128, 128, seed=3)
+    q[0, 0, 1] = -k[0, 0, 1] * 6.0
+    check_against_oracle(Case(1, 256, 256, 2, 2, 128, 128, dtype=dtype, inputs=(q, k, v)))
+
+
+@pytest.mark.parametrize("dtype", DTYPES)
 def test_tiny_workload(dtype):
     w = workloads.get("tiny")
     c = Case(w.B, w.S, w.S, w.Hq, w.Hkv, w.dqk, w.dv, dtype=dtype, inputs=workloads.make_inputs(w))
