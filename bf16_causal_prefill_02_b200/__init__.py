@@ -65,6 +65,10 @@ def _load():
     lib.zq_attn_fwd_debug.restype = i32
     lib.zq_quantize_fp8.argtypes = [P, i32, i64, i32, i32, P, P, P, P]
     lib.zq_quantize_fp8.restype = i32
+    lib.zq_quantize_fp8_noalloc.argtypes = [P, i32, i64, i32, i32, P, P, P]
+    lib.zq_quantize_fp8_noalloc.restype = i32
+    lib.zq_quantize_noalloc_scratch_bytes.argtypes = []
+    lib.zq_quantize_noalloc_scratch_bytes.restype = ctypes.c_size_t
     lib.zq_quantize_workspace_bytes.argtypes = []
     lib.zq_quantize_workspace_bytes.restype = ctypes.c_size_t
     lib.zq_status_string.argtypes = [i32]
@@ -104,6 +108,19 @@ ZQ_DEBUG_BYTES = 128 * 128 * 4 + 128 * 64 * 4 + 256 * 4 + 512 * 12 * 8
 
 def zq_quantize_fp8(x, x_dtype, n_vec, d, hadamard, x_fp8, descale, workspace, stream) -> int:
     return _lib.zq_quantize_fp8(x, x_dtype, n_vec, d, hadamard, x_fp8, descale, workspace, stream)
+
+
+def zq_quantize_fp8_noalloc(x, x_dtype, n_vec, d, hadamard, x_fp8, descale, stream) -> int:
+    """zq_quantize_fp8 without a workspace: for callers that cannot supply
+    device scratch (their device memory belongs to another allocator, or
+    they must not call cudaMalloc in a latency-critical loop).  Uses one
+    fixed scratch array inside the library; calls that overlap on the GPU
+    race.  The first call on a device sets up the array's address."""
+    return _lib.zq_quantize_fp8_noalloc(x, x_dtype, n_vec, d, hadamard, x_fp8, descale, stream)
+
+
+def zq_quantize_noalloc_scratch_bytes() -> int:
+    return int(_lib.zq_quantize_noalloc_scratch_bytes())
 
 
 def zq_quantize_workspace_bytes() -> int:

@@ -135,4 +135,31 @@ cudaError_t launch_quantize(const void* x, int x_bf16, int64_t n, int hadamard, 
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------
+// Allocation-free variant.  Some callers cannot hand the library a device
+// workspace: hosts whose device memory is owned by another allocator that
+// offers no scratch API, and latency-critical serving loops that forbid
+// cudaMalloc because it can synchronise the whole device.  For them the
+// quantiser's scratch (the amax word) lives in a fixed file-scope device
+// array instead.  Every GPU that loads this library keeps the array until
+// the process exits.
+constexpr size_t kNoAllocScratchBytes = 256;
+static __device__ __align__(256) unsigned g_quant_scratch[kNoAllocScratchBytes / sizeof(unsigned)];
+
+// Device address of g_quant_scratch on `dev`, looked up once per device
+// (with that device current) and cached.  nullptr on failure.
+void* noalloc_scratch_for_device(int dev) {
+  constexpr int kMaxDevices = 64;
+  static void* cache[kMaxDevices] = {};
+  if (dev < 0 || dev >= kMaxDevices) return nullptr;
+  void* p = __atomic_load_n(&cache[dev], __ATOMIC_ACQUIRE);
+  if (p) return p;
+  void* ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, g_quant_scratch) != cudaSuccess || !ptr) return nullptr;
+  __atomic_store_n(&cache[dev], ptr, __ATOMIC_RELEASE);
+  return ptr;
+}
+
+size_t noalloc_scratch_capacity() { return kNoAllocScratchBytes; }
+
 }  // namespace zq

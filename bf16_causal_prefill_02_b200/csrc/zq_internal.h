@@ -38,5 +38,7 @@ struct AttnLaunch {
 cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t st);
 cudaError_t launch_quantize(const void* x, int x_bf16, int64_t n, int hadamard, void* out,
                             float* descale, void* workspace, cudaStream_t st, int num_sms);
+void* noalloc_scratch_for_device(int dev);
+size_t noalloc_scratch_capacity();
 
 }  // namespace zq

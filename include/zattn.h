@@ -170,6 +170,35 @@ ZQ_API int zq_quantize_fp8(const void* x, int x_dtype, int64_t n_vec, int d, int
 /* Bytes of device scratch zq_quantize_fp8 needs (a small constant). */
 ZQ_API size_t zq_quantize_workspace_bytes(void);
 
+/*
+ * zq_quantize_fp8_noalloc -- zq_quantize_fp8 without a workspace argument.
+ * (The pages describe no counterpart; this is a library convenience.)
+ *
+ * For callers that cannot provide device scratch memory: hosts whose device
+ * memory belongs to another allocator that offers no scratch API, and
+ * latency-critical loops that must not call cudaMalloc because it can
+ * synchronise the device.  The scratch lives instead in one fixed device
+ * array inside this library, zq_quantize_noalloc_scratch_bytes() bytes
+ * (256), which every GPU that loads the library holds until the process
+ * exits.  The quantiser needs 256 bytes whatever the input size, so every
+ * input the regular entry point accepts fits; a request for more scratch
+ * than the array holds is rejected with ZQ_ERR_SHAPE.
+ *
+ * Arguments, outputs and the other errors are those of zq_quantize_fp8.
+ * The call allocates nothing (no cudaMalloc / cudaFree or allocating library
+ * routine).  The first call on each device looks up the array's device
+ * address with that device current and caches it; make that first call
+ * before any stream capture.  All calls share the one array and it keeps the
+ * last call's contents (the amax word is cleared at the start of each call),
+ * so calls whose work can overlap on the GPU -- on different streams without
+ * ordering between them -- race and must not be issued that way.
+ */
+ZQ_API int zq_quantize_fp8_noalloc(const void* x, int x_dtype, int64_t n_vec, int d, int hadamard,
+                                   void* x_fp8, float* descale, void* stream);
+
+/* Capacity in bytes of the fixed scratch array of zq_quantize_fp8_noalloc. */
+ZQ_API size_t zq_quantize_noalloc_scratch_bytes(void);
+
 /* Static text for a status code (never NULL). */
 ZQ_API const char* zq_status_string(int status);
 
