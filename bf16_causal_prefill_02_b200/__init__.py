@@ -61,7 +61,7 @@ def _load():
     lib.zq_attn_fwd.restype = i32
     lib.zq_attn_fwd_ex.argtypes = [ctypes.POINTER(zq_attn_args), P]
     lib.zq_attn_fwd_ex.restype = i32
-    lib.zq_attn_fwd_debug.argtypes = [ctypes.POINTER(zq_attn_args), P, i32, i32, P]
+    lib.zq_attn_fwd_debug.argtypes = [ctypes.POINTER(zq_attn_args), P, i32, i32, i32, P]
     lib.zq_attn_fwd_debug.restype = i32
     lib.zq_quantize_fp8.argtypes = [P, i32, i64, i32, i32, P, P, P, P]
     lib.zq_quantize_fp8.restype = i32
@@ -69,6 +69,8 @@ def _load():
     lib.zq_quantize_fp8_noalloc.restype = i32
     lib.zq_quantize_noalloc_scratch_bytes.argtypes = []
     lib.zq_quantize_noalloc_scratch_bytes.restype = ctypes.c_size_t
+    lib.zq_debug_exp2.argtypes = [P, P, i64, i32, P]
+    lib.zq_debug_exp2.restype = i32
     lib.zq_quantize_workspace_bytes.argtypes = []
     lib.zq_quantize_workspace_bytes.restype = ctypes.c_size_t
     lib.zq_status_string.argtypes = [i32]
@@ -99,11 +101,11 @@ def zq_attn_fwd_ex(args: zq_attn_args, stream) -> int:
     return _lib.zq_attn_fwd_ex(ctypes.byref(args), stream)
 
 
-def zq_attn_fwd_debug(args: zq_attn_args, dbg, dbg_bh, dbg_qtile, stream) -> int:
-    return _lib.zq_attn_fwd_debug(ctypes.byref(args), dbg, dbg_bh, dbg_qtile, stream)
+def zq_attn_fwd_debug(args: zq_attn_args, dbg, dbg_bh, dbg_qtile, flags, stream) -> int:
+    return _lib.zq_attn_fwd_debug(ctypes.byref(args), dbg, dbg_bh, dbg_qtile, flags, stream)
 
 
-ZQ_DEBUG_BYTES = 128 * 128 * 4 + 128 * 64 * 4 + 256 * 4 + 512 * 12 * 8
+ZQ_DEBUG_BYTES = 128 * 128 * 4 + 128 * 64 * 4 + 256 * 4 + 512 * 16 * 8
 
 
 def zq_quantize_fp8(x, x_dtype, n_vec, d, hadamard, x_fp8, descale, workspace, stream) -> int:
@@ -121,6 +123,10 @@ def zq_quantize_fp8_noalloc(x, x_dtype, n_vec, d, hadamard, x_fp8, descale, stre
 
 def zq_quantize_noalloc_scratch_bytes() -> int:
     return int(_lib.zq_quantize_noalloc_scratch_bytes())
+
+
+def zq_debug_exp2(x, y, n, degree, stream) -> int:
+    return _lib.zq_debug_exp2(x, y, n, degree, stream)
 
 
 def zq_quantize_workspace_bytes() -> int:
@@ -190,7 +196,8 @@ def quantize_fp8(x, hadamard: bool = False, out=None, descale=None, workspace=No
 
 def attn_fwd(q, k, v, out=None, lse=None, softmax_scale=None, causal=True, q_descale=None,
              k_descale=None, v_descale=None, softmax_mode=ZQ_SOFTMAX_LEANP, block_scale=True,
-             headroom_T=8, status=None, return_lse=True, stream=None, debug=None, debug_at=(0, 0)):
+             headroom_T=8, status=None, return_lse=True, stream=None, debug=None, debug_at=(0, 0),
+             debug_flags=0):
     """Causal prefill attention on CUDA tensors.
 
     q (B,Sq,Hq,d_qk), k (B,Sk,Hkv,d_qk), v (B,Sk,Hkv,d_v): bfloat16, or FP8
@@ -224,8 +231,8 @@ def attn_fwd(q, k, v, out=None, lse=None, softmax_scale=None, causal=True, q_des
     a.headroom_T = int(headroom_T)
     a.status = _ptr(status)
     if debug is not None:
-        _check(zq_attn_fwd_debug(a, debug.data_ptr(), int(debug_at[0]), int(debug_at[1]), _stream(stream)),
-               "zq_attn_fwd_debug")
+        _check(zq_attn_fwd_debug(a, debug.data_ptr(), int(debug_at[0]), int(debug_at[1]), int(debug_flags),
+                                 _stream(stream)), "zq_attn_fwd_debug")
     else:
         _check(zq_attn_fwd_ex(a, _stream(stream)), "zq_attn_fwd_ex")
     return out, lse

@@ -23,10 +23,12 @@
 //   S0 [0,128) S1 [128,256)   score tiles; P (bf16x2 or 4 x e4m3 per word)
 //                             is written over the first columns of its S
 //   O  [256,256+DV)           output accumulator
-//   RS [384,400)              FP8: rounded row sum (P times a ones matrix)
+//   RS [384,400)              FP8: rounded row sum (P times the ones block)
 //   SFA [400,408)             FP8: UE8M0 scales of P, one 4-column set per S
 //                             buffer (replicated layout, see sf_smem below)
-//   SFB [408,412)             FP8: scales of V / ones, all 2^0
+//   SFB [408,416)             FP8: scales of V and of the ones block, all 2^0
+// FP8's rounded row sum is the PV MMA run with N = d_v + 16 against V and a
+// block of ones, so it lands in TMEM columns 384..399 right after O.
 // MMA issue order: QK_0, QK_1, PV_0, QK_2, PV_1, ... so the softmax of tile
 // j+1 overlaps PV_j and QK_{j+2}.
 #include <cuda_fp8.h>
@@ -60,14 +62,21 @@ struct Geo {
   static constexpr int VCH = DV * ES / 128;                // 128-byte N chunks of V
   static constexpr int QK_STEPS = QROW / 32;               // 32 bytes of K per MMA
   static constexpr int PV_STEPS = DT == 0 ? 8 : 4;         // 16 (bf16) / 32 (fp8) keys per MMA
-  static constexpr int NS = DT == 0 ? 2 : 4;               // K and V ring stages
+  // K/V ring stages: as many as fit in 227 KB of shared memory
+  static constexpr int NS = DT == 1 ? 4 : (DQK == 128 ? 3 : 2);
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + QBYTES;
   static constexpr int OFF_V = OFF_K + NS * KBYTES;
-  static constexpr int OFF_ONES = OFF_V + NS * VBYTES;     // 16 x 128 keys e4m3, K-major
-  static constexpr int OFF_SF = OFF_ONES + 2048;           // [2 buf][128] scale words
-  static constexpr int OFF_BAR = OFF_SF + 1024;
-  static constexpr int NBAR = 1 + 2 * NS + 2 + 2 + 2 + 1;
+  // FP8: one 128-key x 128-byte block of e4m3 ones after the V stages.  The
+  // PV MMA runs with N = d_v + 16 and reaches it as the second 128-column
+  // atom of V (leading byte offset = ONES - V stage), so the rounded row sum
+  // lands in O's columns d_v .. d_v + 15.
+  static constexpr int ONES_BYTES = DT == 1 ? 16384 : 0;
+  static constexpr int OFF_ONES = OFF_V + NS * VBYTES;
+  static constexpr int OFF_SF = OFF_ONES + ONES_BYTES;     // FP8: [2 buf] 512 B scale tiles
+  static constexpr int SF_BYTES = DT == 1 ? 1024 : 0;
+  static constexpr int OFF_BAR = OFF_SF + SF_BYTES;
+  static constexpr int NBAR = 1 + 2 * NS + 2 + 2 + 1;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;  // + alignment slack
   static_assert(QBYTES % 1024 == 0 && VBYTES % 1024 == 0, "1 KB aligned tiles");
 };
@@ -95,6 +104,46 @@ __device__ __forceinline__ void ffma2(float& r0, float& r1, float a0, float a1, 
       : "=f"(r0), "=f"(r1)
       : "f"(a0), "f"(a1), "f"(b), "f"(c));
 }
+// Software 2^z for a pair of values (offloads the MUFU unit).  Cody-Waite
+// style reduction z = n + f with n = rne(z) (magic-constant add) and
+// f in [-1/2, 1/2], a minimax polynomial p(f) ~ 2^f fitted by the Remez
+// exchange (bf16_causal_prefill_02_b200/csrc/exp2_poly_fit.py; max relative
+// error 7.5e-5 for degree 3, 2.7e-6 for degree 4), and 2^n applied by adding
+// n to the exponent bits.  z is clamped at -126 first (results below 2^-126
+// are irrelevant here: they round to 0 in e4m3 and vanish against the row
+// sum in bf16).
+template <int DEG>
+__device__ __forceinline__ void exp2_poly_x2(float& r0, float& r1, float z0, float z1) {
+  z0 = fmaxf(z0, -126.0f);
+  z1 = fmaxf(z1, -126.0f);
+  const float magic = 12582912.0f;  // 1.5 * 2^23
+  float t0, t1, f0, f1, p0, p1;
+  asm("{\n\t.reg .b64 z, t, n, m;\n\t"
+      "mov.b64 z, {%4, %5};\n\tmov.b64 m, {%6, %6};\n\t"
+      "add.rn.f32x2 t, z, m;\n\tsub.rn.f32x2 n, t, m;\n\tsub.rn.f32x2 z, z, n;\n\t"
+      "mov.b64 {%0, %1}, t;\n\tmov.b64 {%2, %3}, z;\n\t}"
+      : "=f"(t0), "=f"(t1), "=f"(f0), "=f"(f1)
+      : "f"(z0), "f"(z1), "f"(magic));
+  if constexpr (DEG == 3) {
+    ffma2(p0, p1, f0, f1, 5.517166853e-02f, 2.426111251e-01f);
+    asm("{\n\t.reg .b64 p, f, c;\n\tmov.b64 p, {%0, %1};\n\tmov.b64 f, {%2, %3};\n\t"
+        "mov.b64 c, {%4, %4};\n\tfma.rn.f32x2 p, p, f, c;\n\tmov.b64 c, {%5, %5};\n\t"
+        "fma.rn.f32x2 p, p, f, c;\n\tmov.b64 {%0, %1}, p;\n\t}"
+        : "+f"(p0), "+f"(p1)
+        : "f"(f0), "f"(f1), "f"(6.932609677e-01f), "f"(9.999280572e-01f));
+  } else {
+    ffma2(p0, p1, f0, f1, 9.570102207e-03f, 5.591785908e-02f);
+    asm("{\n\t.reg .b64 p, f, c;\n\tmov.b64 p, {%0, %1};\n\tmov.b64 f, {%2, %3};\n\t"
+        "mov.b64 c, {%4, %4};\n\tfma.rn.f32x2 p, p, f, c;\n\tmov.b64 c, {%5, %5};\n\t"
+        "fma.rn.f32x2 p, p, f, c;\n\tmov.b64 c, {%6, %6};\n\tfma.rn.f32x2 p, p, f, c;\n\t"
+        "mov.b64 {%0, %1}, p;\n\t}"
+        : "+f"(p0), "+f"(p1)
+        : "f"(f0), "f"(f1), "f"(2.402474433e-01f), "f"(6.931217909e-01f), "f"(9.999992847e-01f));
+  }
+  r0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  r1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   uint32_t d;
   asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
@@ -136,16 +185,16 @@ __device__ __forceinline__ int next_ref(int eref_old, int emax, int thr) {
 }
 
 
-// Debug trace (clock64 of the traced CTA), per key tile j, 12 slots:
+// Debug trace (clock64 of the traced CTA), per key tile j, 16 slots:
 //   [0] row 0 saw S_j  [1] row 0 loaded S_j  [2] row 0 computed P_j
 //   [3] row 0 released P_j  [4] row 96 released P_j
 //   MMA thread: [5] K_j landed, QK_j issue starts  [6] QK_j issued+committed
 //   [7] P_j seen  [8] V_j landed, PV_j issue starts  [9] PV_j MMAs issued
-//   [10] PV_j committed
+//   [10] PV_j committed  [11..15] unused
 // Lives after the S/P/SF dump in the debug buffer.
 constexpr int kTraceOffsetWords = 128 * 128 + 128 * 64 + 256;
 constexpr int kTraceTiles = 512;
-constexpr int kTraceSlots = 12;
+constexpr int kTraceSlots = 16;
 
 __device__ __forceinline__ uint64_t clk64() {
   uint64_t t;
@@ -173,14 +222,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bar_kvdone = bar_kvfull + G::NS;  // [NS]
   uint64_t* bar_sfull = bar_kvdone + G::NS;   // [2]
   uint64_t* bar_pfull = bar_sfull + 2;        // [2]
-  uint64_t* bar_sf = bar_pfull + 2;           // [2] FP8: scale words staged
-  uint64_t* bar_ofinal = bar_sf + 2;          // [1] last PV landed
+  uint64_t* bar_ofinal = bar_pfull + 2;       // [1] last PV landed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + G::NBAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  // FP8 scale words [buf][row], transposed through shared memory into the
-  // replicated TMEM layout the block-scaled MMA reads: query row r's word
-  // (byte k scales keys 32k..32k+31 of the tile) sits in TMEM column r/32 of
-  // the buffer's 4-column set, at lanes r%32 + 32q of every lane quarter q.
+  // FP8 scale factors staged for tcgen05.cp: per S buffer a 32-row x
+  // 16-byte tile; query row r puts its word at byte 16*(r%32) + 4*(r/32),
+  // and the copy lands it in TMEM column r/32 of the buffer's 4-column set at
+  // lanes r%32 + 32q of every lane quarter q -- the replicated layout the
+  // block-scaled MMA reads.  Byte k of the word scales keys 32k..32k+31.
   uint32_t* sf_smem = reinterpret_cast<uint32_t*>(smem + G::OFF_SF);
 
   const int warp = threadIdx.x >> 5;
@@ -211,7 +260,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar_sfull + s, 1);
       mbar_init(bar_pfull + s, kSoftmaxThreads);
-      mbar_init(bar_sf + s, kSoftmaxThreads);
     }
     mbar_init(bar_ofinal, 1);
     *abort_flag = 0;
@@ -219,7 +267,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (DT == 1) {  // ones operand for the rounded row sum: e4m3 1.0 = 0x38
     uint32_t* ones = reinterpret_cast<uint32_t*>(smem + G::OFF_ONES);
-    for (int i = threadIdx.x; i < 512; i += kThreads) ones[i] = 0x38383838u;
+    for (int i = threadIdx.x; i < G::ONES_BYTES / 4; i += kThreads) ones[i] = 0x38383838u;
     fence_proxy_async_smem();
   }
   if (warp == kWarpMma) {
@@ -280,13 +328,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     // One thread; tcgen05.mma issue runs nearly in step with execution, so
     // this loop is on the critical path: descriptors are built once, each
     // tile costs one K/V wait, one P wait and two commits.
-    if (lane == 0 && n_kv > 0) {
+    if (lane == 0 && n_kv > 0 && !(p.dbg_flags & 1)) {  // flag 1: withhold all work (test hook)
       const uint32_t sbase = smem_u32(smem);
       constexpr uint32_t idesc_qk = idesc_dense(DT == 0 ? 1u : 0u, 0u, 128, 128);
       constexpr uint32_t idesc_pv_bf16 = idesc_dense(1u, 1u, 128, DV);
       // descriptors of stage 0; stage s adds its byte offset >> 4 to the
       // 14-bit start-address field (all addresses stay below 256 KB)
-      uint64_t dq[G::QK_STEPS], dk[G::QK_STEPS], dvv[G::PV_STEPS], d1[4];
+      uint64_t dq[G::QK_STEPS], dk[G::QK_STEPS], dvv[G::PV_STEPS];
 #pragma unroll
       for (int kk = 0; kk < G::QK_STEPS; ++kk) {
         const int pos = kk * 32;
@@ -299,9 +347,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int kk = 0; kk < G::PV_STEPS; ++kk)  // 16 (bf16) or 32 (fp8) keys of V per step
         dvv[kk] = smem_desc(sbase + G::OFF_V + kk * (DT == 0 ? 16 : 32) * 128, 16384, 1024, SW_128B);
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        d1[kk] = smem_desc(sbase + G::OFF_ONES + kk * 32, 16, 1024, SW_128B);
+      // FP8: the second N atom (the ones block) sits at ONES - V_s, so the
+      // descriptor's leading-offset field differs per stage (see voff below)
       auto issue_qk = [&](int j) -> bool {
         const int s = j % G::NS;
         if (!mbar_wait(bar_kvfull + s, (j / G::NS) & 1, lim, abort_flag)) return false;
@@ -325,8 +372,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(bar_pfull + (j & 1), (j >> 1) & 1, lim, abort_flag)) return false;
         tc_fence_after();
         if (trace && j < kTraceTiles) trace[j * kTraceSlots + 8] = clk64();
-        const uint64_t voff = (uint64_t)((s * G::VBYTES) >> 4);
+        uint64_t voff = (uint64_t)((s * G::VBYTES) >> 4);
+        if (DT == 1) {  // replace LBO 16384 by ONES - V_s (both fit the 14-bit field)
+          const uint32_t lbo = (uint32_t)(G::OFF_ONES - (G::OFF_V + s * G::VBYTES));
+          voff += ((uint64_t)(lbo >> 4) << 16) - ((uint64_t)(16384u >> 4) << 16);
+        }
         const uint32_t aP = tbase + kColS0 + (j & 1) * 128;
+        if (DT == 1 && BS)
+          tmem_cp_32x128b_x4(tbase + kColSFA + (j & 1) * 4,
+                             smem_desc(sbase + G::OFF_SF + (j & 1) * 512, 16, 128, SW_NONE));
 #pragma unroll
         for (int kk = 0; kk < G::PV_STEPS; ++kk) {
           const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
@@ -335,12 +389,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_f16_ts(tbase + kColO, aP + kk * 8, dvv[kk] + voff, idesc_pv_bf16, acc);
           } else {
             // 32 keys per step = 8 columns of 4 x e4m3; scale byte kk
+            // N = d_v + 16: V and the ones block in one instruction
             const uint32_t sfa = (tbase + kColSFA + (j & 1) * 4) | ((uint32_t)kk << 30);
             const uint32_t sfb = (tbase + kColSFB) | ((uint32_t)kk << 30);
-            mma_mxf8_ts(tbase + kColO, aP + kk * 8, dvv[kk] + voff, idesc_mx(1u, 128, DV, kk, kk),
-                        sfa, sfb, acc);
-            mma_mxf8_ts(tbase + kColRS, aP + kk * 8, d1[kk], idesc_mx(0u, 128, 16, kk, kk), sfa, sfb,
-                        acc);
+            mma_mxf8_ts(tbase + kColO, aP + kk * 8, dvv[kk] + voff,
+                        idesc_mx(1u, 128, DV + 16, kk, kk), sfa, sfb, acc);
           }
         }
         if (trace && j < kTraceTiles) trace[j * kTraceSlots + 9] = clk64();
@@ -373,6 +426,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       c = ((p.softmax_scale * qd) * kd) * 1.4426950408889634f;
       // SFB (scales of V and of the ones matrix): all 2^0 = 0x7F
       tmem_st4(tbase + lane_off + kColSFB, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+      tmem_st4(tbase + lane_off + kColSFB + 4, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
       if (!BS) {  // running mode: every block scale is 2^0 as well
         tmem_st4(tbase + lane_off + kColSFA, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
         tmem_st4(tbase + lane_off + kColSFA + 4, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
@@ -455,10 +509,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         float lp0 = 0.0f, lp1 = 0.0f;
 #pragma unroll
         for (int cc = 0; cc < 128; cc += 2) {
-          float z0, z1;
+          float z0, z1, p0, p1;
           ffma2(z0, z1, s[cc], s[cc + 1], c, nb);
-          const float p0 = ex2_approx(z0);
-          const float p1 = ex2_approx(z1);
+          if ((cc & 6) == 0) {  // a quarter of the pairs on the FMA pipe
+            exp2_poly_x2<3>(p0, p1, z0, z1);
+          } else {
+            p0 = ex2_approx(z0);
+            p1 = ex2_approx(z1);
+          }
           lp0 += p0;
           lp1 += p1;
           pk[cc / 2] = pack_bf16x2(p0, p1);
@@ -519,11 +577,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float ne = blk == 0 ? (v0 ? -(float)e0 : 0.0f) : (v1 ? -(float)e1 : 0.0f);
 #pragma unroll
             for (int cc = blk * 64; cc < blk * 64 + 64; cc += 4) {
-              float z0, z1, z2, z3;
+              float z0, z1, z2, z3, p0, p1;
               ffma2(z0, z1, s[cc], s[cc + 1], c, ne);
               ffma2(z2, z3, s[cc + 2], s[cc + 3], c, ne);
-              pk[cc / 4] =
-                  pack_e4m3x4(ex2_approx(z0), ex2_approx(z1), ex2_approx(z2), ex2_approx(z3));
+              exp2_poly_x2<4>(p0, p1, z0, z1);  // half of the values on the FMA pipe
+              pk[cc / 4] = pack_e4m3x4(p0, p1, ex2_approx(z2), ex2_approx(z3));
             }
           }
         } else {
@@ -556,13 +614,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int sf1 = v1 ? min(max(e1 - eref + 127, 0), 254) : 0;
         const uint32_t sfw = (uint32_t)sf0 * 0x0101u | ((uint32_t)sf1 * 0x0101u) << 16;
         if (BS) {
-          sf_smem[buf * 128 + row] = sfw;
-          mbar_arrive(bar_sf + buf);
-          w = mbar_wait(bar_sf + buf, (j >> 1) & 1, lim, abort_flag);
-          if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
-          tmem_st4(tbase + lane_off + kColSFA + buf * 4, sf_smem[buf * 128 + lane],
-                   sf_smem[buf * 128 + 32 + lane], sf_smem[buf * 128 + 64 + lane],
-                   sf_smem[buf * 128 + 96 + lane]);
+          sf_smem[buf * 128 + (row & 31) * 4 + (row >> 5)] = sfw;
+          fence_proxy_async_smem();
         }
         if (dump) {
           uint32_t* dp = static_cast<uint32_t*>(p.dbg) + 128 * 128;
@@ -597,7 +650,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld_wait();
           L = __uint_as_float(rs);
         }
-        const bool empty = !(L > 0.0f);
+        // no visible key: L == 0 (FP8), or the reference never left -inf (BF16;
+        // the software exp2 maps masked scores to ~2^-126 instead of 0)
+        const bool empty = !(L > 0.0f) || (DT == 0 && yref == -INFINITY);
         const float inv = empty ? 0.0f : vscale / L;
         if (!empty) {
           const float ref = DT == 0 ? yref : (float)eref;
@@ -637,6 +692,37 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tbase, kTmemCols);
   }
+}
+
+// Evaluates the software exp2 (degree 3 or 4), CUDA's exp2f (degree 0) or
+// the MUFU ex2.approx (degree -1) elementwise, for the test of the polynomial.
+__global__ void exp2_check_kernel(const float* __restrict__ x, float* __restrict__ y, int64_t n,
+                                  int degree) {
+  const int64_t i0 = 2 * ((int64_t)blockIdx.x * blockDim.x + threadIdx.x);
+  if (i0 >= n) return;
+  const float a = x[i0], b = i0 + 1 < n ? x[i0 + 1] : 0.0f;
+  float r0, r1;
+  if (degree == 3) {
+    exp2_poly_x2<3>(r0, r1, a, b);
+  } else if (degree == 4) {
+    exp2_poly_x2<4>(r0, r1, a, b);
+  } else if (degree == 0) {
+    r0 = exp2f(a);
+    r1 = exp2f(b);
+  } else {
+    r0 = ex2_approx(a);
+    r1 = ex2_approx(b);
+  }
+  y[i0] = r0;
+  if (i0 + 1 < n) y[i0 + 1] = r1;
+}
+
+cudaError_t launch_exp2_check(const float* x, float* y, int64_t n, int degree, cudaStream_t st) {
+  const int64_t pairs = (n + 1) / 2;
+  const unsigned blocks = (unsigned)((pairs + 255) / 256);
+  if (blocks == 0) return cudaSuccess;
+  exp2_check_kernel<<<blocks, 256, 0, st>>>(x, y, n, degree);
+  return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------ host side

@@ -75,6 +75,63 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
   }
 }
 
+// True in exactly one lane of the (fully active) warp.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.u32 %0, 1, 0, P;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
+// Non-blocking probe of a phase (never suspends the warp).
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar_addr, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar_addr), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Polling wait that never suspends inside mbarrier.try_wait: test_wait plus
+// an optional nanosleep back-off (sleep_ns = 0: tight spin).
+__device__ __forceinline__ bool mbar_wait_poll(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
+                                               volatile int* abort, uint32_t sleep_ns) {
+  const uint32_t a = smem_u32(bar);
+  if (mbar_test_wait(a, parity)) return true;
+  uint64_t t0 = globaltimer_ns();
+  for (uint32_t n = 1;; ++n) {
+    if (sleep_ns) __nanosleep(sleep_ns);
+    if (mbar_test_wait(a, parity)) return true;
+    if ((n & 255) == 0) {
+      if (*abort) return false;
+      if (globaltimer_ns() - t0 > limit_ns) return false;
+    }
+  }
+}
+
+// Wait variant for the single-issuer roles (TMA producer, MMA issuer), which
+// share an SM sub-partition with a softmax warp: after a failed poll the
+// warp sleeps `sleep_ns`, so waiting costs the softmax warp few issue slots.
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
+                                                volatile int* abort, uint32_t sleep_ns) {
+  const uint32_t a = smem_u32(bar);
+  if (mbar_try_wait(a, parity)) return true;
+  uint64_t t0 = globaltimer_ns();
+  for (uint32_t n = 1;; ++n) {
+    __nanosleep(sleep_ns);
+    if (mbar_try_wait(a, parity)) return true;
+    if ((n & 63) == 0) {
+      if (*abort) return false;
+      if (globaltimer_ns() - t0 > limit_ns) return false;
+    }
+  }
+}
+
 // ------------------------------------------------------------------- fences
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -97,6 +154,24 @@ __device__ __forceinline__ void tma_load_4d(void* smem_dst, const void* desc, ui
       " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(smem_u32(smem_dst)),
       "l"(reinterpret_cast<uint64_t>(desc)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
       : "memory");
+}
+
+// ----------------------------------------------------------- named barriers
+// Barrier `id` (1..15; 0 is __syncthreads) over `nthreads` threads, a
+// multiple of 32, every warp arriving as a whole.
+// bar_red_or returns the OR of `v` over all participating threads.
+__device__ __forceinline__ bool bar_red_or(int id, int nthreads, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\tsetp.ne.u32 pi, %1, 0;\n\t"
+      "bar.red.or.pred po, %2, %3, pi;\n\tselp.u32 %0, 1, 0, po;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ void bar_sync_n(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 // ------------------------------------------------------------ tcgen05 basics

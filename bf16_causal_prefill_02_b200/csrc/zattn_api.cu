@@ -82,7 +82,8 @@ const char* zq_status_string(int s) {
   }
 }
 
-static int attn_impl(const zq_attn_args* a, void* dbg, int dbg_bh, int dbg_t, void* stream) {
+static int attn_impl(const zq_attn_args* a, void* dbg, int dbg_bh, int dbg_t, int dbg_flags,
+                     void* stream) {
   int rc = validate_attn(a);
   if (rc != ZQ_OK) return rc;
   rc = check_device(nullptr);
@@ -116,15 +117,20 @@ static int attn_impl(const zq_attn_args* a, void* dbg, int dbg_bh, int dbg_t, vo
   L.p.dbg = dbg;
   L.p.dbg_bh = dbg_bh;
   L.p.dbg_t = dbg_t;
+  L.p.dbg_flags = dbg_flags;
   cudaError_t e = zq::launch_attention(L, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? ZQ_OK : ZQ_ERR_CUDA;
 }
 
-int zq_attn_fwd_ex(const zq_attn_args* a, void* stream) { return attn_impl(a, nullptr, 0, 0, stream); }
+int zq_attn_fwd_ex(const zq_attn_args* a, void* stream) {
+  return attn_impl(a, nullptr, 0, 0, 0, stream);
+}
 
-int zq_attn_fwd_debug(const zq_attn_args* a, void* dbg, int dbg_bh, int dbg_qtile, void* stream) {
+int zq_attn_fwd_debug(const zq_attn_args* a, void* dbg, int dbg_bh, int dbg_qtile, int flags,
+                      void* stream) {
   if (!dbg) return ZQ_ERR_NULL;
-  return attn_impl(a, dbg, dbg_bh, dbg_qtile, stream);
+  if (flags & ~1) return ZQ_ERR_UNSUPPORTED;
+  return attn_impl(a, dbg, dbg_bh, dbg_qtile, flags, stream);
 }
 
 int zq_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B,
@@ -202,5 +208,15 @@ int zq_quantize_fp8_noalloc(const void* x, int x_dtype, int64_t n_vec, int d, in
 }
 
 size_t zq_quantize_noalloc_scratch_bytes(void) { return zq::noalloc_scratch_capacity(); }
+
+int zq_debug_exp2(const float* x, float* y, int64_t n, int degree, void* stream) {
+  if (n < 0) return ZQ_ERR_SHAPE;
+  if (n > 0 && (!x || !y)) return ZQ_ERR_NULL;
+  if (degree != 3 && degree != 4 && degree != 0 && degree != -1) return ZQ_ERR_UNSUPPORTED;
+  int rc = check_device(nullptr);
+  if (rc != ZQ_OK) return rc;
+  cudaError_t e = zq::launch_exp2_check(x, y, n, degree, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ZQ_OK : ZQ_ERR_CUDA;
+}
 
 }  // extern "C"

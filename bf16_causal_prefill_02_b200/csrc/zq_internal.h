@@ -25,6 +25,11 @@ struct AttnParams {
   // scale words here: float S[128][128]; uint32 P[128][64]; uint32 SF[2][128].
   void* dbg;
   int dbg_bh, dbg_t;
+  // Test hook: bit 0 makes the MMA issuer withhold all work, so every other
+  // role's wait runs into its time limit and the kernel reports
+  // ZQ_ERR_TIMEOUT through the status word (exercises the failure path
+  // without faulting or hanging the GPU).
+  int dbg_flags;
 };
 
 struct AttnLaunch {
@@ -39,6 +44,7 @@ cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t st);
 cudaError_t launch_quantize(const void* x, int x_bf16, int64_t n, int hadamard, void* out,
                             float* descale, void* workspace, cudaStream_t st, int num_sms);
 void* noalloc_scratch_for_device(int dev);
+cudaError_t launch_exp2_check(const float* x, float* y, int64_t n, int degree, cudaStream_t st);
 size_t noalloc_scratch_capacity();
 
 }  // namespace zq

@@ -136,11 +136,15 @@ ZQ_API int zq_attn_fwd_ex(const zq_attn_args* args, void* stream);
  * scale), uint32 P[128][64] (bf16: 64 words of 2 x bf16; FP8: the first 32
  * words hold 4 x e4m3 each, key order little-endian), uint32 SF[2][128]
  * (FP8: the UE8M0 scale of 64-key block 0 / 1 of each row, repeated in all
- * four bytes), then uint64 TRACE[512][12]: SM clock (clock64) at twelve points of
- * the pipeline for key tile j (see attn_fwd.cu).  For tests and tuning. */
-#define ZQ_DEBUG_BYTES (128 * 128 * 4 + 128 * 64 * 4 + 256 * 4 + 512 * 12 * 8)
+ * four bytes), then uint64 TRACE[512][16]: SM clock (clock64) at up to sixteen points of
+ * the pipeline for key tile j (see attn_fwd.cu).  flags: 0, or 1 to make
+ * the MMA issuer withhold all work so that every other role's bounded wait
+ * runs out: the kernel then writes ZQ_ERR_TIMEOUT to args->status and
+ * returns (about two seconds later) with the outputs undefined; nothing
+ * faults or hangs.  For tests and tuning. */
+#define ZQ_DEBUG_BYTES (128 * 128 * 4 + 128 * 64 * 4 + 256 * 4 + 512 * 16 * 8)
 ZQ_API int zq_attn_fwd_debug(const zq_attn_args* args, void* dbg, int dbg_bh, int dbg_qtile,
-                             void* stream);
+                             int flags, void* stream);
 
 /*
  * zq_quantize_fp8 -- per-tensor FP8 e4m3 quantiser with an optional fused
@@ -198,6 +202,14 @@ ZQ_API int zq_quantize_fp8_noalloc(const void* x, int x_dtype, int64_t n_vec, in
 
 /* Capacity in bytes of the fixed scratch array of zq_quantize_fp8_noalloc. */
 ZQ_API size_t zq_quantize_noalloc_scratch_bytes(void);
+
+/* zq_debug_exp2 -- y[i] = 2^x[i] by the kernels' software exp2 (degree 3 or
+ * 4 minimax polynomial after range reduction), by CUDA's exp2f (degree 0) or
+ * by the hardware approximation ex2.approx (degree -1).  x, y: device fp32
+ * arrays of n elements.  For the test that bounds the polynomial's error
+ * against exp2f.  Errors: ZQ_ERR_SHAPE, ZQ_ERR_NULL, ZQ_ERR_UNSUPPORTED,
+ * ZQ_ERR_ARCH, ZQ_ERR_CUDA. */
+ZQ_API int zq_debug_exp2(const float* x, float* y, int64_t n, int degree, void* stream);
 
 /* Static text for a status code (never NULL). */
 ZQ_API const char* zq_status_string(int status);

@@ -159,6 +159,22 @@ def test_bitwise_deterministic(dtype):
         assert torch.equal(l.view(torch.int32), l0.view(torch.int32))
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "leanp"])
+def test_timeout_path_reports_status_and_context_survives(dtype):
+    # The MMA issuer withholds all work (test hook): every other role's
+    # bounded wait runs out, the kernel writes ZQ_ERR_TIMEOUT and returns.
+    import bf16_causal_prefill_02_b200 as zq
+
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    dbg = torch.zeros(zq.ZQ_DEBUG_BYTES // 4, dtype=torch.int32, device="cuda")
+    c = Case(1, 256, 256, 1, 1, 128, 128, dtype=dtype, seed=4)
+    c.run_gpu(debug=dbg, status=st, debug_flags=1)
+    torch.cuda.synchronize()
+    assert int(st.item()) == zq.ZQ_ERR_TIMEOUT
+    # the context is still usable and a normal launch is correct
+    check_against_oracle(Case(1, 256, 256, 1, 1, 128, 128, dtype=dtype, seed=4))
+
+
 def test_status_word_stays_zero():
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     c = Case(1, 256, 256, 2, 2, 128, 128, dtype="leanp", seed=1)
