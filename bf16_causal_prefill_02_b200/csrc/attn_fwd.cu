@@ -16,12 +16,18 @@
 //        "How ZYFA works" (scaling by powers of 2 before rounding).
 //
 // One CTA computes one 128-row query tile of one (batch, head).  Warp roles:
-//   warps 0-3  softmax + epilogue; thread t owns query row t (TMEM lane t)
-//   warp 4     TMA producer (Q once, then K/V tiles through an NS-stage ring)
-//   warp 5     TMEM allocator and single-thread tcgen05.mma issuer
+//   warps 0-7  softmax + epilogue.  TMEM lane quarter q (query rows
+//              32q..32q+31) belongs to warps q and q+4, 16 rows each; inside
+//              a warp, threads t and t+16 share a row, thread t taking keys
+//              0-63 of every tile and thread t+16 keys 64-127 (one 64-key
+//              scale block each; 16x32bx2 TMEM accesses)
+//   warp 8     TMA producer (Q once, then K/V tiles through an NS-stage ring)
+//   warp 9     TMEM allocator and tcgen05 issuer (the whole warp runs the
+//              loop, one elected lane issues)
 // Tensor memory (512 columns x 128 lanes, fp32 words):
-//   S0 [0,128) S1 [128,256)   score tiles; P (bf16x2 or 4 x e4m3 per word)
-//                             is written over the first columns of its S
+//   S0 [0,128) S1 [128,256)   score tiles; P (bf16x2 or 4 x e4m3 per word) of
+//                             keys 64h..64h+63 is written over the first
+//                             columns of S half h (column 64h onwards)
 //   O  [256,256+DV)           output accumulator
 //   RS [384,400)              FP8: rounded row sum (P times the ones block)
 //   SFA [400,408)             FP8: UE8M0 scales of P, one 4-column set per S
@@ -43,9 +49,9 @@
 namespace zq {
 
 constexpr int kTile = 128;
-constexpr int kSoftmaxThreads = 128;
+constexpr int kSoftmaxThreads = 256;
 constexpr int kThreads = kSoftmaxThreads + 64;
-constexpr int kWarpProducer = 4, kWarpMma = 5;
+constexpr int kWarpProducer = 8, kWarpMma = 9;
 constexpr uint32_t kColS0 = 0, kColO = 256, kColRS = 384, kColSFA = 400, kColSFB = 408;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kInvalidExp = -(1 << 20);
@@ -78,6 +84,8 @@ struct Geo {
   static constexpr int OFF_BAR = OFF_SF + SF_BYTES;
   static constexpr int NBAR = 1 + 2 * NS + 2 + 2 + 1;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;  // + alignment slack
+  static_assert(SMEM <= 232448, "227 KB of shared memory per CTA");
+  static_assert(DV == 128, "the two halves of a row split d_v = 128 in 64 + 64");
   static_assert(QBYTES % 1024 == 0 && VBYTES % 1024 == 0, "1 KB aligned tiles");
 };
 
@@ -187,10 +195,13 @@ __device__ __forceinline__ int next_ref(int eref_old, int emax, int thr) {
 
 // Debug trace (clock64 of the traced CTA), per key tile j, 16 slots:
 //   [0] row 0 saw S_j  [1] row 0 loaded S_j  [2] row 0 computed P_j
-//   [3] row 0 released P_j  [4] row 96 released P_j
-//   MMA thread: [5] K_j landed, QK_j issue starts  [6] QK_j issued+committed
-//   [7] P_j seen  [8] V_j landed, PV_j issue starts  [9] PV_j MMAs issued
-//   [10] PV_j committed  [11..15] unused
+//   [3] warp 0 released P_j  [4] warp 3 released P_j
+//   [11] warp 1 released P_j  [12] warp 5 released P_j (warps 1 and 5 share
+//        their SM sub-partition with the MMA warp)
+//   MMA warp: [5] K_j landed, QK_j issue starts  [13] two QK_j MMAs issued
+//   [6] QK_j issued + committed  [7] P_j seen  [8] block scales copied
+//   [14] two PV_j MMAs issued  [9] PV_j MMAs issued  [10] PV_j committed
+//   [15] unused
 // Lives after the S/P/SF dump in the debug buffer.
 constexpr int kTraceOffsetWords = 128 * 128 + 128 * 64 + 256;
 constexpr int kTraceTiles = 512;
@@ -202,7 +213,7 @@ __device__ __forceinline__ uint64_t clk64() {
   return t;
 }
 
-template <int DT, int DQK, int DV, int MODE, int BS>
+template <int DT, int DQK, int DV, int MODE, int BS, int DBG>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQ2,
                     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmK2,
@@ -247,7 +258,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int max_key = p.causal ? min(q1 + shift, p.Sk - 1) : p.Sk - 1;
   const int n_kv = max_key < 0 ? 0 : max_key / kTile + 1;
   const int min_lim = p.causal ? min(q0 + shift, p.Sk - 1) : p.Sk - 1;
-  const bool traced = p.dbg != nullptr && t == p.dbg_t && bh == p.dbg_bh;
+  // debug dumps and the trace exist only in the DBG instantiation
+  const bool traced = DBG && p.dbg != nullptr && t == p.dbg_t && bh == p.dbg_bh;
   uint64_t* trace = traced ? reinterpret_cast<uint64_t*>(static_cast<uint32_t*>(p.dbg) + kTraceOffsetWords)
                            : nullptr;
 
@@ -325,10 +337,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
-    // One thread; tcgen05.mma issue runs nearly in step with execution, so
-    // this loop is on the critical path: descriptors are built once, each
-    // tile costs one K/V wait, one P wait and two commits.
-    if (lane == 0 && n_kv > 0 && !(p.dbg_flags & 1)) {  // flag 1: withhold all work (test hook)
+    // tcgen05.mma issue runs nearly in step with execution, so this loop is
+    // on the critical path.  The whole warp runs it, so that descriptors and
+    // control stay warp-uniform; one elected lane issues every tcgen05 op
+    // (the same lane each time: elect.sync picks the lowest active lane).
+    if (n_kv > 0 && !(DBG && (p.dbg_flags & 1))) {  // flag 1: withhold all work (test hook)
       const uint32_t sbase = smem_u32(smem);
       constexpr uint32_t idesc_qk = idesc_dense(DT == 0 ? 1u : 0u, 0u, 128, 128);
       constexpr uint32_t idesc_pv_bf16 = idesc_dense(1u, 1u, 128, DV);
@@ -347,168 +360,204 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int kk = 0; kk < G::PV_STEPS; ++kk)  // 16 (bf16) or 32 (fp8) keys of V per step
         dvv[kk] = smem_desc(sbase + G::OFF_V + kk * (DT == 0 ? 16 : 32) * 128, 16384, 1024, SW_128B);
+      auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
+        return __all_sync(0xffffffffu, mbar_wait(bar, parity, lim, abort_flag));
+      };
       // FP8: the second N atom (the ones block) sits at ONES - V_s, so the
       // descriptor's leading-offset field differs per stage (see voff below)
       auto issue_qk = [&](int j) -> bool {
         const int s = j % G::NS;
-        if (!mbar_wait(bar_kvfull + s, (j / G::NS) & 1, lim, abort_flag)) return false;
+        if (!wait_all(bar_kvfull + s, (j / G::NS) & 1)) return false;
         tc_fence_after();
-        if (trace && j < kTraceTiles) trace[j * kTraceSlots + 5] = clk64();
+        if (trace && lane == 0 && j < kTraceTiles) trace[j * kTraceSlots + 5] = clk64();
         const uint32_t dS = tbase + kColS0 + (j & 1) * 128;
         const uint64_t koff = (uint64_t)((s * G::KBYTES) >> 4);
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < G::QK_STEPS; ++kk) {
-          if (DT == 0)
-            mma_f16_ss(dS, dq[kk], dk[kk] + koff, idesc_qk, kk > 0);
-          else
-            mma_f8_ss(dS, dq[kk], dk[kk] + koff, idesc_qk, kk > 0);
+          for (int kk = 0; kk < G::QK_STEPS; ++kk) {
+            if (DT == 0)
+              mma_f16_ss(dS, dq[kk], dk[kk] + koff, idesc_qk, kk > 0);
+            else
+              mma_f8_ss(dS, dq[kk], dk[kk] + koff, idesc_qk, kk > 0);
+            if (trace && kk == 1 && j < kTraceTiles) trace[j * kTraceSlots + 13] = clk64();
+          }
+          tc_commit(bar_sfull + (j & 1));
         }
-        tc_commit(bar_sfull + (j & 1));
-        if (trace && j < kTraceTiles) trace[j * kTraceSlots + 6] = clk64();
+        __syncwarp();
+        if (trace && lane == 0 && j < kTraceTiles) trace[j * kTraceSlots + 6] = clk64();
         return true;
       };
       auto issue_pv = [&](int j) -> bool {
         const int s = j % G::NS;
-        if (!mbar_wait(bar_pfull + (j & 1), (j >> 1) & 1, lim, abort_flag)) return false;
+        if (!wait_all(bar_pfull + (j & 1), (j >> 1) & 1)) return false;
         tc_fence_after();
-        if (trace && j < kTraceTiles) trace[j * kTraceSlots + 8] = clk64();
+        if (trace && lane == 0 && j < kTraceTiles) trace[j * kTraceSlots + 7] = clk64();
         uint64_t voff = (uint64_t)((s * G::VBYTES) >> 4);
         if (DT == 1) {  // replace LBO 16384 by ONES - V_s (both fit the 14-bit field)
           const uint32_t lbo = (uint32_t)(G::OFF_ONES - (G::OFF_V + s * G::VBYTES));
           voff += ((uint64_t)(lbo >> 4) << 16) - ((uint64_t)(16384u >> 4) << 16);
         }
+        // P of keys [64h, 64h + 64) sits at the start of S half h
         const uint32_t aP = tbase + kColS0 + (j & 1) * 128;
-        if (DT == 1 && BS)
-          tmem_cp_32x128b_x4(tbase + kColSFA + (j & 1) * 4,
-                             smem_desc(sbase + G::OFF_SF + (j & 1) * 512, 16, 128, SW_NONE));
+        if (elect_one()) {
+          if (DT == 1 && BS)
+            tmem_cp_32x128b_x4(tbase + kColSFA + (j & 1) * 4,
+                               smem_desc(sbase + G::OFF_SF + (j & 1) * 512, 16, 128, SW_NONE));
+          if (trace && j < kTraceTiles) trace[j * kTraceSlots + 8] = clk64();
 #pragma unroll
-        for (int kk = 0; kk < G::PV_STEPS; ++kk) {
-          const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
-          if (DT == 0) {
-            // 16 keys per step = 8 packed bf16x2 columns of P
-            mma_f16_ts(tbase + kColO, aP + kk * 8, dvv[kk] + voff, idesc_pv_bf16, acc);
-          } else {
-            // 32 keys per step = 8 columns of 4 x e4m3; scale byte kk
-            // N = d_v + 16: V and the ones block in one instruction
-            const uint32_t sfa = (tbase + kColSFA + (j & 1) * 4) | ((uint32_t)kk << 30);
-            const uint32_t sfb = (tbase + kColSFB) | ((uint32_t)kk << 30);
-            mma_mxf8_ts(tbase + kColO, aP + kk * 8, dvv[kk] + voff,
-                        idesc_mx(1u, 128, DV + 16, kk, kk), sfa, sfb, acc);
+          for (int kk = 0; kk < G::PV_STEPS; ++kk) {
+            const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
+            if (DT == 0) {
+              // 16 keys per step = 8 packed bf16x2 columns of P
+              mma_f16_ts(tbase + kColO, aP + (kk >> 2) * 64 + (kk & 3) * 8, dvv[kk] + voff, idesc_pv_bf16, acc);
+            } else {
+              // 32 keys per step = 8 columns of 4 x e4m3; scale byte kk
+              // N = d_v + 16: V and the ones block in one instruction
+              const uint32_t sfa = (tbase + kColSFA + (j & 1) * 4) | ((uint32_t)kk << 30);
+              const uint32_t sfb = (tbase + kColSFB) | ((uint32_t)kk << 30);
+              mma_mxf8_ts(tbase + kColO, aP + (kk >> 1) * 64 + (kk & 1) * 8, dvv[kk] + voff,
+                          idesc_mx(1u, 128, DV + 16, kk, kk), sfa, sfb, acc);
+            }
+            if (trace && kk == 1 && j < kTraceTiles) trace[j * kTraceSlots + 14] = clk64();
           }
+          if (trace && j < kTraceTiles) trace[j * kTraceSlots + 9] = clk64();
+          tc_commit(bar_kvdone + s);
         }
-        if (trace && j < kTraceTiles) trace[j * kTraceSlots + 9] = clk64();
-        tc_commit(bar_kvdone + s);
-        if (trace && j < kTraceTiles) trace[j * kTraceSlots + 10] = clk64();
+        __syncwarp();
+        if (trace && lane == 0 && j < kTraceTiles) trace[j * kTraceSlots + 10] = clk64();
         return true;
       };
-      bool ok = true;
-      if (!mbar_wait(bar_q, 0, lim, abort_flag)) ok = false;
+      bool ok = wait_all(bar_q, 0);
       for (int j = 0; ok && j < n_kv; ++j) {
         if (!issue_qk(j)) { ok = false; break; }
         if (j > 0 && !issue_pv(j - 1)) { ok = false; break; }
       }
       if (ok && !issue_pv(n_kv - 1)) ok = false;
-      if (ok) tc_commit(bar_ofinal);
-      if (!ok) fail();
+      if (ok && elect_one()) tc_commit(bar_ofinal);
+      __syncwarp();
+      if (!ok && lane == 0) fail();
     }
   } else {
     // ------------------------------------------------------ softmax (rows)
-    const int row = threadIdx.x;  // query row == TMEM lane
+    // Warps q and q + 4 share TMEM lane quarter q: warp q owns lanes
+    // 32q..32q+15 and warp q + 4 lanes 32q+16..32q+31 (16x32bx2 accesses).
+    // Inside a warp, threads t and t + 16 own the same query row: thread t
+    // takes keys [0, 64) of every tile, thread t + 16 keys [64, 128) -- one
+    // 64-key scale block each -- and the two agree on the row's reference
+    // with one shuffle.  P of keys [64h, 64h + 64) goes over the first
+    // columns of S half h, which only this thread pair reads.
+    const int qd = warp & 3, sub = warp >> 2;
+    const int half = lane >> 4;
+    const int row = qd * 32 + sub * 16 + (lane & 15);  // query row == TMEM lane
+    const uint32_t col_h = (uint32_t)half * 64;
     const int i = q0 + row;
     const int row_lim = p.causal ? min(i + shift, p.Sk - 1) : p.Sk - 1;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const uint32_t lane_off = (uint32_t)(qd * 32 + sub * 16) << 16;  // 16-lane group
+    constexpr unsigned kFull = 0xffffffffu;
     float c = p.softmax_scale * 1.4426950408889634f;  // log2(e)
     float vscale = 1.0f;
     if (DT == 1) {
-      const float qd = p.q_descale ? *p.q_descale : 1.0f;
-      const float kd = p.k_descale ? *p.k_descale : 1.0f;
+      const float qds = p.q_descale ? *p.q_descale : 1.0f;
+      const float kds = p.k_descale ? *p.k_descale : 1.0f;
       vscale = p.v_descale ? *p.v_descale : 1.0f;
-      c = ((p.softmax_scale * qd) * kd) * 1.4426950408889634f;
-      // SFB (scales of V and of the ones matrix): all 2^0 = 0x7F
-      tmem_st4(tbase + lane_off + kColSFB, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
-      tmem_st4(tbase + lane_off + kColSFB + 4, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
-      if (!BS) {  // running mode: every block scale is 2^0 as well
-        tmem_st4(tbase + lane_off + kColSFA, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
-        tmem_st4(tbase + lane_off + kColSFA + 4, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+      c = ((p.softmax_scale * qds) * kds) * 1.4426950408889634f;
+      if (sub == 0) {
+        // SFB (scales of V and of the ones matrix): all 2^0 = 0x7F; warp q
+        // writes all 32 lanes of its quarter
+        const uint32_t q_off = (uint32_t)(qd * 32) << 16;
+        tmem_st4(tbase + q_off + kColSFB, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+        tmem_st4(tbase + q_off + kColSFB + 4, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+        if (!BS) {  // running mode: every block scale is 2^0 as well
+          tmem_st4(tbase + q_off + kColSFA, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+          tmem_st4(tbase + q_off + kColSFA + 4, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+        }
+        tmem_st_wait();
       }
-      tmem_st_wait();
     }
     const int T = p.headroom_T;
     float yref = -INFINITY;   // BF16 / FP8 running mode: log2-domain reference
     int eref = kInvalidExp;   // FP8: reference exponent E (invalid until a key is seen)
-    float l = 0.0f;           // BF16 row sum (fp32, unrounded p)
+    float l = 0.0f;           // BF16: this thread's half of the row sum (fp32, unrounded p)
     bool ok = true;
+
+    // O holds tiles < j at the old reference: rescale this thread's 64 O
+    // columns by f once PV_{j-1} has landed (rare: the reference is lazy)
+    auto rescale_o = [&](int j, float f) -> bool {
+      const bool w2 = mbar_wait(bar_kvdone + (j - 1) % G::NS, ((j - 1) / G::NS) & 1, lim, abort_flag);
+      if (!__all_sync(kFull, w2)) return false;
+      tc_fence_after();
+#pragma unroll 1
+      for (int ch = 0; ch < 2; ++ch) {
+        uint32_t o[32];
+        const uint32_t to = tbase + lane_off + kColO + ch * 32;
+        tmem_ld16x2_32<64>(to, o);
+        tmem_ld_wait();
+#pragma unroll
+        for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * f);
+        tmem_st16x2_32<64>(to, o);
+      }
+      if (DT == 1) {
+        // all 16 row-sum columns hold the same sum: half 0 keeps column RS,
+        // half 1 column RS + 1
+        uint32_t rs;
+        tmem_ld16x2_1<1>(tbase + lane_off + kColRS, rs);
+        tmem_ld_wait();
+        tmem_st16x2_1<1>(tbase + lane_off + kColRS, __float_as_uint(__uint_as_float(rs) * f));
+      }
+      return true;
+    };
 
     for (int j = 0; ok && j < n_kv; ++j) {
       const int buf = j & 1;
-      bool w = mbar_wait(bar_sfull + buf, (j >> 1) & 1, lim, abort_flag);
-      if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+      const bool w = mbar_wait(bar_sfull + buf, (j >> 1) & 1, lim, abort_flag);
+      if (!__all_sync(kFull, w)) { ok = false; break; }
       tc_fence_after();
-      if (trace && row == 0 && j < kTraceTiles) trace[j * kTraceSlots + 0] = clk64();
-      float s[128];  // explicit bit casts: no type punning through pointers
+      if (trace && warp == 0 && lane == 0 && j < kTraceTiles) trace[j * kTraceSlots + 0] = clk64();
+      float s[64];  // explicit bit casts: no type punning through pointers
       {
-        uint32_t a0[32], a1[32], a2[32], a3[32];
+        uint32_t a0[32], a1[32];
         const uint32_t ts = tbase + lane_off + kColS0 + buf * 128;
-        tmem_ld32(ts, a0);
-        tmem_ld32(ts + 32, a1);
-        tmem_ld32(ts + 64, a2);
-        tmem_ld32(ts + 96, a3);
+        tmem_ld16x2_32<64>(ts, a0);
+        tmem_ld16x2_32<64>(ts + 32, a1);
         tmem_ld_wait();
 #pragma unroll
         for (int cc = 0; cc < 32; ++cc) {
           s[cc] = __uint_as_float(a0[cc]);
           s[32 + cc] = __uint_as_float(a1[cc]);
-          s[64 + cc] = __uint_as_float(a2[cc]);
-          s[96 + cc] = __uint_as_float(a3[cc]);
         }
       }
-      if (trace && row == 0 && j < kTraceTiles) trace[j * kTraceSlots + 1] = clk64();
+      if (trace && warp == 0 && lane == 0 && j < kTraceTiles) trace[j * kTraceSlots + 1] = clk64();
       const bool dump = traced && j == 0;
       if (dump) {
-        float* ds = static_cast<float*>(p.dbg) + row * 128;
+        float* ds = static_cast<float*>(p.dbg) + row * 128 + col_h;
 #pragma unroll
-        for (int cc = 0; cc < 128; ++cc) ds[cc] = s[cc];
+        for (int cc = 0; cc < 64; ++cc) ds[cc] = s[cc];
       }
-      const int kbase = j * kTile;
-      if (kbase + kTile - 1 > min_lim) {
+      const int kbase = j * kTile + (int)col_h;
+      if (kbase + 63 > min_lim) {
 #pragma unroll
-        for (int cc = 0; cc < 128; ++cc)
+        for (int cc = 0; cc < 64; ++cc)
           if (kbase + cc > row_lim) s[cc] = -INFINITY;
       }
-      const float m0 = max64(s), m1 = max64(s + 64);  // raw block maxima
+      const float m = max64(s);  // raw block maximum
       const uint32_t tP = tbase + lane_off + kColS0 + buf * 128;
 
       if constexpr (DT == 0) {
         // ------------------------------------------------ BF16, exact exp2
-        const float ymax = fmaxf(m0, m1) * c;
-        const bool need = ymax > yref + 8.0f;
-        if (__any_sync(0xffffffffu, need)) {
+        const float ym = m * c;
+        const float ymax = fmaxf(ym, __shfl_xor_sync(kFull, ym, 16));  // the row's maximum
+        if (__builtin_expect(__any_sync(kFull, ymax > yref + 8.0f), 0)) {
           const float nref = fmaxf(yref, ymax);
           const float f = (nref == -INFINITY || yref == nref) ? 1.0f : ex2_approx(yref - nref);
           yref = nref;
           l *= f;
-          if (j > 0) {
-            // O holds tiles < j; PV_{j-1} must have landed before rescaling
-            w = mbar_wait(bar_kvdone + (j - 1) % G::NS, ((j - 1) / G::NS) & 1, lim, abort_flag);
-            if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
-            tc_fence_after();
-#pragma unroll 1
-            for (int ch = 0; ch < DV / 32; ++ch) {
-              uint32_t o[32];
-              const uint32_t to = tbase + lane_off + kColO + ch * 32;
-              tmem_ld32(to, o);
-              tmem_ld_wait();
-#pragma unroll
-              for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * f);
-              tmem_st32(to, o);
-            }
-          }
+          if (j > 0 && !rescale_o(j, f)) { ok = false; break; }
         }
         const float nb = yref == -INFINITY ? 0.0f : -yref;
-        uint32_t pk[64];
+        uint32_t pk[32];
         float lp0 = 0.0f, lp1 = 0.0f;
 #pragma unroll
-        for (int cc = 0; cc < 128; cc += 2) {
+        for (int cc = 0; cc < 64; cc += 2) {
           float z0, z1, p0, p1;
           ffma2(z0, z1, s[cc], s[cc + 1], c, nb);
           if ((cc & 6) == 0) {  // a quarter of the pairs on the FMA pipe
@@ -522,133 +571,114 @@ __global__ void __launch_bounds__(kThreads, 1)
           pk[cc / 2] = pack_bf16x2(p0, p1);
         }
         l += lp0 + lp1;
-        if (trace && row == 0 && j < kTraceTiles) trace[j * kTraceSlots + 2] = clk64();
-        tmem_st32(tP, *reinterpret_cast<uint32_t(*)[32]>(pk));
-        tmem_st32(tP + 32, *reinterpret_cast<uint32_t(*)[32]>(pk + 32));
+        if (trace && warp == 0 && lane == 0 && j < kTraceTiles) trace[j * kTraceSlots + 2] = clk64();
+        tmem_st16x2_32<64>(tP, pk);
         if (dump) {
           uint32_t* dp = static_cast<uint32_t*>(p.dbg) + 128 * 128;
 #pragma unroll
-          for (int q = 0; q < 64; ++q) dp[row * 64 + q] = pk[q];
+          for (int q = 0; q < 32; ++q) dp[row * 64 + half * 32 + q] = pk[q];
         }
       } else {
         // ------------------------------------------------ FP8 P path
-        int e0, e1;  // block exponents of keys [0,64) and [64,128)
-        int nref;
+        // e: this thread's block exponent; the row's reference E (eref)
+        // moves only when a block exceeds it by more than 32 (block scale),
+        // or follows the running maximum (running mode: one exponent per row)
+        int e, nref;
         if (BS) {
-          e0 = m0 != -INFINITY ? (int)ceilf(m0 * c) - T : kInvalidExp;
-          e1 = m1 != -INFINITY ? (int)ceilf(m1 * c) - T : kInvalidExp;
-          nref = next_ref(eref, max(e0, e1), 32);
+          e = m != -INFINITY ? (int)ceilf(m * c) - T : kInvalidExp;
+          nref = next_ref(eref, max(e, __shfl_xor_sync(kFull, e, 16)), 32);
         } else {
-          // running mode: one exponent from the running max of the row
-          yref = fmaxf(fmaxf(m0, m1) * c, yref);
+          const float ym = m * c;
+          yref = fmaxf(yref, fmaxf(ym, __shfl_xor_sync(kFull, ym, 16)));
           nref = yref != -INFINITY ? (int)ceilf(yref) - T : kInvalidExp;
-          e0 = e1 = nref;
+          e = nref;  // the row's exponent for both blocks
         }
         const bool grow = eref > kInvalidExp && nref != eref;
-        if (j > 0 && __any_sync(0xffffffffu, grow)) {
-          // O and the row sum hold tiles < j at scale 2^(-eref): move them to
-          // 2^(-nref) exactly.  PV_{j-1} must have landed first.
-          const float f = grow ? pow2i(max(eref - nref, -126)) : 1.0f;
-          w = mbar_wait(bar_kvdone + (j - 1) % G::NS, ((j - 1) / G::NS) & 1, lim, abort_flag);
-          if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
-          tc_fence_after();
-#pragma unroll 1
-          for (int ch = 0; ch < DV / 32; ++ch) {
-            uint32_t o[32];
-            const uint32_t to = tbase + lane_off + kColO + ch * 32;
-            tmem_ld32(to, o);
-            tmem_ld_wait();
-#pragma unroll
-            for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * f);
-            tmem_st32(to, o);
-          }
-          uint32_t rs;
-          tmem_ld1(tbase + lane_off + kColRS, rs);
-          tmem_ld_wait();
-          tmem_st1(tbase + lane_off + kColRS, __float_as_uint(__uint_as_float(rs) * f));
+        if (__builtin_expect(j > 0 && __any_sync(kFull, grow), 0)) {
+          // O and the row sum hold tiles < j at scale 2^(-eref): move them
+          // to 2^(-nref) exactly
+          if (!rescale_o(j, grow ? pow2i(max(eref - nref, -126)) : 1.0f)) { ok = false; break; }
         }
         eref = nref;
-        const bool v0 = e0 > kInvalidExp, v1 = e1 > kInvalidExp;
-        uint32_t pk[32];
+        const bool v = e > kInvalidExp;
+        uint32_t pk[16];
         if (MODE == 0) {
           // exact: e4m3_rne(exp2(y - e))
+          const float ne = v ? -(float)e : 0.0f;
 #pragma unroll
-          for (int blk = 0; blk < 2; ++blk) {
-            const float ne = blk == 0 ? (v0 ? -(float)e0 : 0.0f) : (v1 ? -(float)e1 : 0.0f);
-#pragma unroll
-            for (int cc = blk * 64; cc < blk * 64 + 64; cc += 4) {
-              float z0, z1, z2, z3, p0, p1;
-              ffma2(z0, z1, s[cc], s[cc + 1], c, ne);
-              ffma2(z2, z3, s[cc + 2], s[cc + 3], c, ne);
-              exp2_poly_x2<4>(p0, p1, z0, z1);  // half of the values on the FMA pipe
-              pk[cc / 4] = pack_e4m3x4(p0, p1, ex2_approx(z2), ex2_approx(z3));
-            }
+          for (int cc = 0; cc < 64; cc += 4) {
+            float z0, z1, z2, z3, p0, p1;
+            ffma2(z0, z1, s[cc], s[cc + 1], c, ne);
+            ffma2(z2, z3, s[cc + 2], s[cc + 3], c, ne);
+            exp2_poly_x2<4>(p0, p1, z0, z1);  // half of the values on the FMA pipe
+            pk[cc / 4] = pack_e4m3x4(p0, p1, ex2_approx(z2), ex2_approx(z3));
           }
         } else {
           // Lean P: u = sat((8(y - e) + 56) / 128) clamps the code at 0; the
           // magic add 1.5*2^23 rounds 128u half-to-even into the low byte.
           const float a = c * 0.0625f;  // 8c / 128
           const float magic = 12582912.0f;
+          const float k0 = v ? (float)(56 - 8 * e) * 0.0078125f : 0.0f;
 #pragma unroll
-          for (int blk = 0; blk < 2; ++blk) {
-            const int e = blk == 0 ? e0 : e1;
-            const bool v = blk == 0 ? v0 : v1;
-            const float k0 = v ? (float)(56 - 8 * e) * 0.0078125f : 0.0f;
-#pragma unroll
-            for (int cc = blk * 64; cc < blk * 64 + 64; cc += 4) {
-              const float u0 = fma_sat(s[cc], a, k0);
-              const float u1 = fma_sat(s[cc + 1], a, k0);
-              const float u2 = fma_sat(s[cc + 2], a, k0);
-              const float u3 = fma_sat(s[cc + 3], a, k0);
-              float x0, x1, x2, x3;
-              ffma2(x0, x1, u0, u1, 128.0f, magic);
-              ffma2(x2, x3, u2, u3, 128.0f, magic);
-              pk[cc / 4] = prmt(prmt(__float_as_uint(x0), __float_as_uint(x1), 0x0040u),
-                                prmt(__float_as_uint(x2), __float_as_uint(x3), 0x0040u), 0x5410u);
-            }
+          for (int cc = 0; cc < 64; cc += 4) {
+            const float u0 = fma_sat(s[cc], a, k0);
+            const float u1 = fma_sat(s[cc + 1], a, k0);
+            const float u2 = fma_sat(s[cc + 2], a, k0);
+            const float u3 = fma_sat(s[cc + 3], a, k0);
+            float x0, x1, x2, x3;
+            ffma2(x0, x1, u0, u1, 128.0f, magic);
+            ffma2(x2, x3, u2, u3, 128.0f, magic);
+            pk[cc / 4] = prmt(prmt(__float_as_uint(x0), __float_as_uint(x1), 0x0040u),
+                              prmt(__float_as_uint(x2), __float_as_uint(x3), 0x0040u), 0x5410u);
           }
         }
-        if (trace && row == 0 && j < kTraceTiles) trace[j * kTraceSlots + 2] = clk64();
-        tmem_st32(tP, pk);
-        const int sf0 = v0 ? min(max(e0 - eref + 127, 0), 254) : 0;
-        const int sf1 = v1 ? min(max(e1 - eref + 127, 0), 254) : 0;
-        const uint32_t sfw = (uint32_t)sf0 * 0x0101u | ((uint32_t)sf1 * 0x0101u) << 16;
+        if (trace && warp == 0 && lane == 0 && j < kTraceTiles) trace[j * kTraceSlots + 2] = clk64();
+        tmem_st16x2_16<64>(tP, pk);
+        const int sf = v ? min(max(e - eref + 127, 0), 254) : 0;
         if (BS) {
-          sf_smem[buf * 128 + (row & 31) * 4 + (row >> 5)] = sfw;
+          // bytes 2h, 2h+1 of the row's word: K32 chunks 2h and 2h+1
+          reinterpret_cast<uint16_t*>(sf_smem + buf * 128 + (row & 31) * 4 + (row >> 5))[half] =
+              (uint16_t)(sf * 0x0101u);
           fence_proxy_async_smem();
         }
         if (dump) {
           uint32_t* dp = static_cast<uint32_t*>(p.dbg) + 128 * 128;
 #pragma unroll
-          for (int q = 0; q < 32; ++q) dp[row * 64 + q] = pk[q];
-          dp[128 * 64 + row] = (uint32_t)sf0 * 0x01010101u;
-          dp[128 * 64 + 128 + row] = (uint32_t)sf1 * 0x01010101u;
+          for (int q = 0; q < 16; ++q) dp[row * 64 + half * 16 + q] = pk[q];
+          dp[128 * 64 + half * 128 + row] = (uint32_t)sf * 0x01010101u;
         }
       }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar_pfull + buf);
-      if (trace && j < kTraceTiles) {
-        if (row == 0) trace[j * kTraceSlots + 3] = clk64();
-        if (row == 96) trace[j * kTraceSlots + 4] = clk64();
+      if (trace && j < kTraceTiles && lane == 0) {
+        if (warp == 0) trace[j * kTraceSlots + 3] = clk64();
+        if (warp == 3) trace[j * kTraceSlots + 4] = clk64();
+        if (warp == 1) trace[j * kTraceSlots + 11] = clk64();
+        if (warp == 5) trace[j * kTraceSlots + 12] = clk64();
       }
     }
     if (!ok) {
-      fail();
+      if (lane == 0) fail();
     } else {
       // ------------------------------------------------------------ epilogue
-      float L = l, lse_v = -INFINITY;
       bool wok = true;
-      if (n_kv > 0) wok = __all_sync(0xffffffffu, mbar_wait(bar_ofinal, 0, lim, abort_flag));
+      if (n_kv > 0) wok = __all_sync(kFull, mbar_wait(bar_ofinal, 0, lim, abort_flag));
       if (!wok) {
-        fail();
+        if (lane == 0) fail();
       } else {
         tc_fence_after();
-        if (DT == 1 && n_kv > 0) {
-          uint32_t rs;
-          tmem_ld1(tbase + lane_off + kColRS, rs);
-          tmem_ld_wait();
-          L = __uint_as_float(rs);
+        float L, lse_v = -INFINITY;
+        if (DT == 1) {
+          L = 0.0f;
+          if (n_kv > 0) {
+            uint32_t rs;
+            tmem_ld16x2_1<1>(tbase + lane_off + kColRS, rs);  // columns RS / RS + 1: equal
+            tmem_ld_wait();
+            L = __uint_as_float(rs);
+          }
+        } else {
+          L = l + __shfl_xor_sync(kFull, l, 16);  // same value in both halves
         }
         // no visible key: L == 0 (FP8), or the reference never left -inf (BF16;
         // the software exp2 maps masked scores to ~2^-126 instead of 0)
@@ -659,12 +689,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           lse_v = (ref + __log2f(L)) * 0.6931471805599453f;
         }
         __nv_bfloat16* orow =
-            static_cast<__nv_bfloat16*>(p.out) + (((int64_t)b * p.Sq + i) * p.Hq + h) * DV;
+            static_cast<__nv_bfloat16*>(p.out) + (((int64_t)b * p.Sq + i) * p.Hq + h) * DV + col_h;
 #pragma unroll 1
-        for (int ch = 0; ch < DV / 32; ++ch) {
+        for (int ch = 0; ch < 2; ++ch) {
           uint32_t o[32];
           if (n_kv > 0) {
-            tmem_ld32(tbase + lane_off + kColO + ch * 32, o);
+            tmem_ld16x2_32<64>(tbase + lane_off + kColO + ch * 32, o);
             tmem_ld_wait();
           } else {
 #pragma unroll
@@ -681,7 +711,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
           }
         }
-        if (p.lse && i < p.Sq) p.lse[((int64_t)b * p.Hq + h) * p.Sq + i] = lse_v;
+        if (half == 0 && p.lse && i < p.Sq) p.lse[((int64_t)b * p.Hq + h) * p.Sq + i] = lse_v;
       }
     }
   }
@@ -780,7 +810,7 @@ static cudaError_t launch_variant(const AttnLaunch& a, cudaStream_t st) {
     mQ2 = mQ;
     mK2 = mK;
   }
-  auto kern = attn_fwd_kernel<DT, DQK, DV, MODE, BS>;
+  auto kern = p.dbg ? attn_fwd_kernel<DT, DQK, DV, MODE, BS, 1> : attn_fwd_kernel<DT, DQK, DV, MODE, BS, 0>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM);
   if (e != cudaSuccess) return e;
   const long long nblocks = (long long)p.n_qtiles * p.B * p.Hq;
