@@ -276,41 +276,78 @@ def time_steps(fn, steps, warmup, world):
     return max_over_ranks(ms, world)
 
 
+def _oracle_inputs(w, dtype, hadamard):
+    """The kernel's inputs for `w` as fp64 arrays (FP8: quantised and decoded,
+    as the kernel sees them)."""
+    import oracle
+
+    q, k, v = (t.numpy() for t in workloads.make_inputs(w))
+    if dtype == "bf16":
+        return tuple(torch.from_numpy(t).to(torch.bfloat16).double().numpy() for t in (q, k, v))
+    deq = []
+    for t, rot in ((q, hadamard), (k, hadamard), (v, False)):
+        c, d = oracle.quantize_fp8(t, hadamard=rot)
+        deq.append(oracle.dequant_e4m3(c, float(d)))
+    return tuple(deq)
+
+
+def _oracle_rows(w, dtype, qd, kd, vd, rows):
+    """Run the oracle (R1 for bf16, R2 of the mode for FP8) on `rows`;
+    returns the causal FLOPs those rows stand for."""
+    import oracle
+
+    if dtype == "bf16":
+        oracle.attn_ref(qd, kd, vd, rows=rows)
+    else:
+        oracle.attn_fp8_emul(qd, kd, vd, rows=rows,
+                             mode=oracle.MODE_EXACT if dtype == "exact" else oracle.MODE_LEANP)
+    i = rows % w.S
+    return float(np.sum(2.0 * (w.dqk + w.dv) * (i + 1)))
+
+
 def cpu_oracle_rate(w, dtype, seconds, hadamard=False):
     """Time the oracle on host cores over a bounded row sample of `w`.
     Returns (TFLOP/s, cores, sample description)."""
     import oracle
 
-    q, k, v = (t.numpy() for t in workloads.make_inputs(w))
-    if dtype == "bf16":
-        qd, kd, vd = (torch.from_numpy(t).to(torch.bfloat16).double().numpy() for t in (q, k, v))
-    else:
-        deq = []
-        for t, rot in ((q, hadamard), (k, hadamard), (v, False)):
-            c, d = oracle.quantize_fp8(t, hadamard=rot)
-            deq.append(oracle.dequant_e4m3(c, float(d)))
-        qd, kd, vd = deq
-    S = w.S
+    qd, kd, vd = _oracle_inputs(w, dtype, hadamard)
     rng = np.random.default_rng(0)
     done_rows, flops, elapsed = 0, 0.0, 0.0
     batch = 64
     while elapsed < seconds:
-        rows = rng.integers(0, w.B * w.Hq * S, size=batch)
-        i = rows % S
+        rows = rng.integers(0, w.B * w.Hq * w.S, size=batch)
         t0 = time.perf_counter()
-        if dtype == "bf16":
-            oracle.attn_ref(qd, kd, vd, rows=rows)
-        else:
-            oracle.attn_fp8_emul(qd, kd, vd, rows=rows,
-                                 mode=oracle.MODE_EXACT if dtype == "exact" else oracle.MODE_LEANP)
+        f = _oracle_rows(w, dtype, qd, kd, vd, rows)
         elapsed += time.perf_counter() - t0
-        flops += float(np.sum(2.0 * (w.dqk + w.dv) * (i + 1)))
+        flops += f
         done_rows += batch
         batch = min(batch * 2, 4096)
     desc = ("%d uniformly drawn query rows of %s (fp64 %s on kernel inputs; inputs quantised "
             "beforehand, untimed), %.1f s" % (done_rows, w.name,
                                                "R1 exact" if dtype == "bf16" else "R2 " + dtype, elapsed))
     return flops / elapsed / 1e12, oracle.num_threads(), desc
+
+
+def oracle_steps(w, dtype, steps, warmup, rows_per_step, hadamard=False):
+    """The reference arm: `warmup` untimed and `steps` timed oracle steps,
+    each over `rows_per_step` query rows drawn uniformly (seeded) from the
+    workload.  Returns (TFLOP/s, ms per step, cores, sample description)."""
+    import oracle
+
+    qd, kd, vd = _oracle_inputs(w, dtype, hadamard)
+    rng = np.random.default_rng(1)
+    for _ in range(warmup):
+        _oracle_rows(w, dtype, qd, kd, vd, rng.integers(0, w.B * w.Hq * w.S, size=rows_per_step))
+    flops, elapsed = 0.0, 0.0
+    for _ in range(steps):
+        rows = rng.integers(0, w.B * w.Hq * w.S, size=rows_per_step)
+        t0 = time.perf_counter()
+        flops += _oracle_rows(w, dtype, qd, kd, vd, rows)
+        elapsed += time.perf_counter() - t0
+    desc = ("%d timed steps of %d uniformly drawn query rows of %s each (fp64 %s on kernel inputs; "
+            "inputs quantised beforehand, untimed), %.1f s" %
+            (steps, rows_per_step, w.name, "R1 exact" if dtype == "bf16" else "R2 " + dtype, elapsed))
+    return flops / elapsed / 1e12, elapsed / max(steps, 1) * 1e3, oracle.num_threads(), desc
 
 
 def run_ours(args, rank, world, w):
@@ -379,28 +416,31 @@ def run_ours(args, rank, world, w):
 
 def main():
     args = parse()
-    rank, world, local = dist_setup(args.gpus)
     w = workloads.get(args.workload, args.S)
     if args.impl == "reference":
+        # host-only: rank 0 times the oracle, the other ranks exit without
+        # work (no process group, no GPU)
+        rank = int(os.environ.get("RANK", "0"))
         if rank == 0:
-            tf, cores, desc = cpu_oracle_rate(w, args.dtype, args.cpu_seconds * max(1, args.steps) / 40.0,
-                                              args.hadamard)
+            # each step a bounded sample: about 0.1-0.3 s of oracle work at 32K
+            rows = max(32, min(1024, int(256 * 32768 / max(w.S, 1))))
+            tf, ms, cores, desc = oracle_steps(w, args.dtype, args.steps, args.warmup, rows, args.hadamard)
             line = {"impl": "reference", "metric": "causal prefill attention TFLOP/s (FP8, BF16) at "
                     "S=16K/32K; % of B200 tensor peak", "value": tf, "unit": "TFLOP/s",
-                    "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+                    "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
+                    "warmup": args.warmup, "ms_per_step": round(ms, 3),
                     "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                     "dtype": "f64", "data": "synthetic",
-                    "config": {"workload": "%s_%s" % (w.name, args.dtype)},
+                    "config": {"workload": "%s_%s%s" % (w.name, args.dtype, "_hadamard" if args.hadamard else ""),
+                               "B": w.B, "S": w.S, "Hq": w.Hq, "Hkv": w.Hkv, "d_qk": w.dqk, "d_v": w.dv,
+                               "causal": True, "softmax": args.dtype},
                     "cpu_baseline": {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                                      "sample": desc},
                     "e2e": {"value": tf, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                             "d2h_bytes_per_step": 0}}
             print(json.dumps(line), flush=True)
-        if world > 1:
-            import torch.distributed as dist
-
-            dist.destroy_process_group()
         return
+    rank, world, local = dist_setup(args.gpus)
     res = run_ours(args, rank, world, w)
     if rank == 0 and not args.no_cpu:
         tf, cores, desc = cpu_oracle_rate(w, args.dtype, args.cpu_seconds, args.hadamard)

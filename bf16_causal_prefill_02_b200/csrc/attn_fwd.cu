@@ -519,7 +519,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t ts = tbase + lane_off + kColS0 + buf * 128;
         tmem_ld16x2_32<64>(ts, a0);
         tmem_ld16x2_32<64>(ts + 32, a1);
-        tmem_ld_wait();
+        tmem_ld_wait_regs(a0, a1);
 #pragma unroll
         for (int cc = 0; cc < 32; ++cc) {
           s[cc] = __uint_as_float(a0[cc]);
