@@ -246,10 +246,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work unit: longest causal rows first
-  const int BH = p.B * p.Hq;
-  const int t = p.n_qtiles - 1 - (int)(blockIdx.x / BH);
-  const int bh = (int)(blockIdx.x % BH);
+  // ---- work unit: groups of head_group heads; inside a group, longest
+  // causal rows first, interleaved across its heads
+  const int GH = p.head_group;
+  const int gi = (int)(blockIdx.x / ((unsigned)GH * p.n_qtiles));
+  const int gr = (int)(blockIdx.x % ((unsigned)GH * p.n_qtiles));
+  const int t = p.n_qtiles - 1 - gr / GH;
+  const int bh = gi * GH + gr % GH;
   const int b = bh / p.Hq, h = bh % p.Hq;
   const int g = h / (p.Hq / p.Hkv);
   const int q0 = t * kTile;
@@ -610,7 +613,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             float z0, z1, z2, z3, p0, p1;
             ffma2(z0, z1, s[cc], s[cc + 1], c, ne);
             ffma2(z2, z3, s[cc + 2], s[cc + 3], c, ne);
-            exp2_poly_x2<4>(p0, p1, z0, z1);  // half of the values on the FMA pipe
+            if ((cc & 4) == 0) {
+              exp2_poly_x2<4>(p0, p1, z0, z1);  // a quarter of the values on the FMA pipe
+            } else {
+              p0 = ex2_approx(z0);
+              p1 = ex2_approx(z1);
+            }
             pk[cc / 4] = pack_e4m3x4(p0, p1, ex2_approx(z2), ex2_approx(z3));
           }
         } else {

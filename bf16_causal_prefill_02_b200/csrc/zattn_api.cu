@@ -109,6 +109,19 @@ static int attn_impl(const zq_attn_args* a, void* dbg, int dbg_bh, int dbg_t, in
   L.p.Hq = a->Hq;
   L.p.Hkv = a->Hkv;
   L.p.n_qtiles = (a->Sq + 127) / 128;
+  {
+    // Group 4 heads (one K/V head under 4:1 GQA) when the K/V of all heads
+    // is well past what the 126 MB L2 keeps around (96 MB): blocks then
+    // stream shared K/V tiles.
+    // Smaller problems keep longest-rows-first over every head, which
+    // balances the tail better.
+    const int bh = a->B * a->Hq;
+    const double es = a->dtype == ZQ_DTYPE_FP8_E4M3 ? 1.0 : 2.0;
+    const double kv_bytes = (double)a->B * a->Hkv * a->Sk * (a->d_qk + a->d_v) * es;
+    int gh = bh;
+    if (kv_bytes > 96.0 * 1024 * 1024) gh = bh % 4 == 0 ? 4 : (bh % 2 == 0 ? 2 : 1);
+    L.p.head_group = gh;
+  }
   L.p.causal = a->causal ? 1 : 0;
   L.p.headroom_T = a->dtype == ZQ_DTYPE_FP8_E4M3 ? a->headroom_T : 8;
   L.p.softmax_scale =

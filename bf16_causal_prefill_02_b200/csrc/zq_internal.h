@@ -16,6 +16,13 @@ struct AttnParams {
   int* status;
   int B, Sq, Sk, Hq, Hkv;
   int n_qtiles;
+  // Block order: blocks come in groups of head_group consecutive flat heads
+  // (head_group divides B * Hq); inside a group, query tiles run longest
+  // causal rows first, interleaved across the group's heads.  head_group =
+  // B * Hq is plain longest-rows-first over all heads; a small group keeps
+  // the blocks that run together on few heads, so their K/V tiles are
+  // shared in L2.
+  int head_group;
   int causal;
   int headroom_T;
   float softmax_scale;

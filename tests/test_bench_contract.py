@@ -1,0 +1,42 @@
+"""The bench.py contract on the host: the reference arm (the oracle on host
+cores) prints one JSON line with the keys the driver reads, and exits 0 on a
+machine without a GPU; under a multi-rank launch only rank 0 prints."""
+import json
+import os
+import subprocess
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _run(args, env_extra=None):
+    env = dict(os.environ)
+    env.update(env_extra or {})
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py")] + args, cwd=ROOT, env=env,
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    return [json.loads(l) for l in r.stdout.splitlines() if l.startswith("{")]
+
+
+def test_reference_arm_line():
+    lines = _run(["--impl", "reference", "--workload", "tiny", "--steps", "3", "--warmup", "1"])
+    assert len(lines) == 1
+    r = lines[0]
+    assert r["impl"] == "reference"
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e"):
+        assert key in r, key
+    assert r["unit"] == "TFLOP/s" and r["higher_is_better"] is True
+    assert r["steps"] == 3 and r["warmup"] == 1
+    assert r["value"] > 0 and r["cpu_baseline"]["value"] == r["value"]
+    assert r["cpu_baseline"]["kind"] == "oracle" and r["cpu_baseline"]["cores"] >= 1
+    assert r["e2e"] == {"value": r["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+    assert r["config"]["workload"] == "tiny_leanp"
+
+
+def test_reference_arm_other_ranks_are_silent():
+    lines = _run(["--impl", "reference", "--workload", "tiny", "--steps", "2", "--warmup", "1"],
+                 {"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
+    assert lines == []
