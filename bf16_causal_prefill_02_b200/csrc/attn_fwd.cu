@@ -82,7 +82,7 @@ struct Geo {
   static constexpr int OFF_SF = OFF_ONES + ONES_BYTES;     // FP8: [2 buf] 512 B scale tiles
   static constexpr int SF_BYTES = DT == 1 ? 1024 : 0;
   static constexpr int OFF_BAR = OFF_SF + SF_BYTES;
-  static constexpr int NBAR = 1 + 2 * NS + 2 + 2 + 1;
+  static constexpr int NBAR = 1 + 2 * NS + 2 + 2 + 1 + 2;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;  // + alignment slack
   static_assert(SMEM <= 232448, "227 KB of shared memory per CTA");
   static_assert(DV == 128, "the two halves of a row split d_v = 128 in 64 + 64");
@@ -213,7 +213,32 @@ __device__ __forceinline__ uint64_t clk64() {
   return t;
 }
 
-template <int DT, int DQK, int DV, int MODE, int BS, int DBG>
+// One work unit: a 128-row query tile t of flat head bh = batch * Hq + head.
+// Units are numbered in groups of head_group consecutive heads; inside a
+// group, longest causal rows first, interleaved across the group's heads.
+struct Unit {
+  int t, bh, b, h, g, q0, n_kv, min_lim;
+};
+__device__ __forceinline__ Unit unit_of(const AttnParams& p, int u) {
+  Unit w;
+  const int GH = p.head_group;
+  const int gi = u / (GH * p.n_qtiles), gr = u % (GH * p.n_qtiles);
+  w.t = p.n_qtiles - 1 - gr / GH;
+  w.bh = gi * GH + gr % GH;
+  w.b = w.bh / p.Hq;
+  w.h = w.bh % p.Hq;
+  w.g = w.h / (p.Hq / p.Hkv);
+  w.q0 = w.t * kTile;
+  const int q1 = min(w.q0 + kTile - 1, p.Sq - 1);
+  const int shift = p.Sk - p.Sq;
+  const int max_key = p.causal ? min(q1 + shift, p.Sk - 1) : p.Sk - 1;
+  w.n_kv = max_key < 0 ? 0 : max_key / kTile + 1;
+  w.min_lim = p.causal ? min(w.q0 + shift, p.Sk - 1) : p.Sk - 1;
+  return w;
+}
+
+// PERSIST = 0: one unit per CTA (the grid has one CTA per unit).
+template <int DT, int DQK, int DV, int MODE, int BS, int DBG, int PERSIST>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQ2,
                     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmK2,
@@ -233,7 +258,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bar_kvdone = bar_kvfull + G::NS;  // [NS]
   uint64_t* bar_sfull = bar_kvdone + G::NS;   // [2]
   uint64_t* bar_pfull = bar_sfull + 2;        // [2]
-  uint64_t* bar_ofinal = bar_pfull + 2;       // [1] last PV landed
+  uint64_t* bar_ofinal = bar_pfull + 2;       // [1] last PV of a unit landed
+  // A CTA runs units one after another (persistent); the barrier phases run
+  // on across units, every role counting the same sequence of key tiles
+  // (jt) and of units with work (nq).
+  uint64_t* bar_qfree = bar_ofinal + 1;       // [1] last QK of a unit done: Q reusable
+  uint64_t* bar_ofree = bar_qfree + 1;        // [1] softmax read O (and RS) of a unit
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + G::NBAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   // FP8 scale factors staged for tcgen05.cp: per S buffer a 32-row x
@@ -246,25 +276,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work unit: groups of head_group heads; inside a group, longest
-  // causal rows first, interleaved across its heads
-  const int GH = p.head_group;
-  const int gi = (int)(blockIdx.x / ((unsigned)GH * p.n_qtiles));
-  const int gr = (int)(blockIdx.x % ((unsigned)GH * p.n_qtiles));
-  const int t = p.n_qtiles - 1 - gr / GH;
-  const int bh = gi * GH + gr % GH;
-  const int b = bh / p.Hq, h = bh % p.Hq;
-  const int g = h / (p.Hq / p.Hkv);
-  const int q0 = t * kTile;
-  const int q1 = min(q0 + kTile - 1, p.Sq - 1);
+  const int n_units = p.n_qtiles * p.B * p.Hq;
+  // The k-th unit of this CTA: rounds of gridDim.x units, walked forwards in
+  // even rounds and backwards in odd ones, so that under longest-rows-first
+  // numbering every CTA pairs long units with short ones (a plain stride
+  // would hand CTA 0 about twice the work of the last CTA).  Strictly
+  // increasing in k.
+  auto unit_at = [&](int k) -> int {
+    return k * (int)gridDim.x + ((k & 1) ? (int)gridDim.x - 1 - (int)blockIdx.x : (int)blockIdx.x);
+  };
   const int shift = p.Sk - p.Sq;
-  const int max_key = p.causal ? min(q1 + shift, p.Sk - 1) : p.Sk - 1;
-  const int n_kv = max_key < 0 ? 0 : max_key / kTile + 1;
-  const int min_lim = p.causal ? min(q0 + shift, p.Sk - 1) : p.Sk - 1;
   // debug dumps and the trace exist only in the DBG instantiation
-  const bool traced = DBG && p.dbg != nullptr && t == p.dbg_t && bh == p.dbg_bh;
-  uint64_t* trace = traced ? reinterpret_cast<uint64_t*>(static_cast<uint32_t*>(p.dbg) + kTraceOffsetWords)
-                           : nullptr;
+  auto traced_unit = [&](const Unit& w) { return DBG && p.dbg != nullptr && w.t == p.dbg_t && w.bh == p.dbg_bh; };
+  uint64_t* const trace_buf =
+      DBG && p.dbg ? reinterpret_cast<uint64_t*>(static_cast<uint32_t*>(p.dbg) + kTraceOffsetWords) : nullptr;
 
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 1);
@@ -277,6 +302,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar_pfull + s, kSoftmaxThreads);
     }
     mbar_init(bar_ofinal, 1);
+    mbar_init(bar_qfree, 1);
+    mbar_init(bar_ofree, kSoftmaxThreads);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -311,32 +338,42 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == kWarpProducer) {
     // ------------------------------------------------------------ producer
-    if (lane == 0 && n_kv > 0) {
-      uint8_t* sq = smem + G::OFF_Q;
-      mbar_arrive_expect_tx(bar_q, G::QBYTES);
-#pragma unroll
-      for (int c = 0; c < G::NCH; ++c) {
-        const bool narrow = (c == G::NCH - 1) && G::LASTW == 64;
-        tma_load_4d(sq + c * 16384, narrow ? (const void*)&tmQ2 : (const void*)&tmQ, bar_q,
-                    c * 128 / G::ES, h, q0, b);
-      }
-      for (int j = 0; j < n_kv; ++j) {
-        const int s = j % G::NS;
-        const uint32_t ph = ((j / G::NS) & 1) ^ 1;  // first pass through the ring: free
-        if (!mbar_wait(bar_kvdone + s, ph, lim, abort_flag)) { fail(); break; }
-        uint8_t* sk = smem + G::OFF_K + s * G::KBYTES;
-        uint8_t* sv = smem + G::OFF_V + s * G::VBYTES;
-        mbar_arrive_expect_tx(bar_kvfull + s, G::KBYTES + G::VBYTES);
+    if (lane == 0) {
+      int jt = 0, nq = 0;
+      bool ok = true;
+      for (int k = 0, u = unit_at(0); ok && u < n_units; u = PERSIST ? unit_at(++k) : n_units) {
+        const Unit w = unit_of(p, u);
+        if (w.n_kv == 0) continue;
+        // Q of the previous unit is read until its last QK completes
+        if (nq > 0 && !mbar_wait(bar_qfree, (nq - 1) & 1, lim, abort_flag)) { ok = false; break; }
+        uint8_t* sq = smem + G::OFF_Q;
+        mbar_arrive_expect_tx(bar_q, G::QBYTES);
 #pragma unroll
         for (int c = 0; c < G::NCH; ++c) {
           const bool narrow = (c == G::NCH - 1) && G::LASTW == 64;
-          tma_load_4d(sk + c * 16384, narrow ? (const void*)&tmK2 : (const void*)&tmK,
-                      bar_kvfull + s, c * 128 / G::ES, g, j * kTile, b);
+          tma_load_4d(sq + c * 16384, narrow ? (const void*)&tmQ2 : (const void*)&tmQ, bar_q,
+                      c * 128 / G::ES, w.h, w.q0, w.b);
         }
+        for (int j = 0; j < w.n_kv; ++j, ++jt) {
+          const int s = jt % G::NS;
+          const uint32_t ph = ((jt / G::NS) & 1) ^ 1;  // first pass through the ring: free
+          if (!mbar_wait(bar_kvdone + s, ph, lim, abort_flag)) { ok = false; break; }
+          uint8_t* sk = smem + G::OFF_K + s * G::KBYTES;
+          uint8_t* sv = smem + G::OFF_V + s * G::VBYTES;
+          mbar_arrive_expect_tx(bar_kvfull + s, G::KBYTES + G::VBYTES);
 #pragma unroll
-        for (int c = 0; c < G::VCH; ++c)
-          tma_load_4d(sv + c * 16384, &tmV, bar_kvfull + s, c * 128 / G::ES, g, j * kTile, b);
+          for (int c = 0; c < G::NCH; ++c) {
+            const bool narrow = (c == G::NCH - 1) && G::LASTW == 64;
+            tma_load_4d(sk + c * 16384, narrow ? (const void*)&tmK2 : (const void*)&tmK,
+                        bar_kvfull + s, c * 128 / G::ES, w.g, j * kTile, w.b);
+          }
+#pragma unroll
+          for (int c = 0; c < G::VCH; ++c)
+            tma_load_4d(sv + c * 16384, &tmV, bar_kvfull + s, c * 128 / G::ES, w.g, j * kTile, w.b);
+        }
+        ++nq;
       }
+      if (!ok) fail();
     }
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
@@ -344,7 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // on the critical path.  The whole warp runs it, so that descriptors and
     // control stay warp-uniform; one elected lane issues every tcgen05 op
     // (the same lane each time: elect.sync picks the lowest active lane).
-    if (n_kv > 0 && !(DBG && (p.dbg_flags & 1))) {  // flag 1: withhold all work (test hook)
+    if (!(DBG && (p.dbg_flags & 1))) {  // flag 1: withhold all work (test hook)
       const uint32_t sbase = smem_u32(smem);
       constexpr uint32_t idesc_qk = idesc_dense(DT == 0 ? 1u : 0u, 0u, 128, 128);
       constexpr uint32_t idesc_pv_bf16 = idesc_dense(1u, 1u, 128, DV);
@@ -368,12 +405,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       // FP8: the second N atom (the ones block) sits at ONES - V_s, so the
       // descriptor's leading-offset field differs per stage (see voff below)
-      auto issue_qk = [&](int j) -> bool {
-        const int s = j % G::NS;
-        if (!wait_all(bar_kvfull + s, (j / G::NS) & 1)) return false;
+      // jg: the tile's place in the CTA's sequence (stage, buffer, parity);
+      // j: its index inside the unit (accumulate flag, trace slot)
+      uint64_t* trace = nullptr;
+      auto issue_qk = [&](int jg, int j) -> bool {
+        const int s = jg % G::NS;
+        if (!wait_all(bar_kvfull + s, (jg / G::NS) & 1)) return false;
         tc_fence_after();
         if (trace && lane == 0 && j < kTraceTiles) trace[j * kTraceSlots + 5] = clk64();
-        const uint32_t dS = tbase + kColS0 + (j & 1) * 128;
+        const uint32_t dS = tbase + kColS0 + (jg & 1) * 128;
         const uint64_t koff = (uint64_t)((s * G::KBYTES) >> 4);
         if (elect_one()) {
 #pragma unroll
@@ -384,15 +424,15 @@ __global__ void __launch_bounds__(kThreads, 1)
               mma_f8_ss(dS, dq[kk], dk[kk] + koff, idesc_qk, kk > 0);
             if (trace && kk == 1 && j < kTraceTiles) trace[j * kTraceSlots + 13] = clk64();
           }
-          tc_commit(bar_sfull + (j & 1));
+          tc_commit(bar_sfull + (jg & 1));
         }
         __syncwarp();
         if (trace && lane == 0 && j < kTraceTiles) trace[j * kTraceSlots + 6] = clk64();
         return true;
       };
-      auto issue_pv = [&](int j) -> bool {
-        const int s = j % G::NS;
-        if (!wait_all(bar_pfull + (j & 1), (j >> 1) & 1)) return false;
+      auto issue_pv = [&](int jg, int j) -> bool {
+        const int s = jg % G::NS;
+        if (!wait_all(bar_pfull + (jg & 1), (jg >> 1) & 1)) return false;
         tc_fence_after();
         if (trace && lane == 0 && j < kTraceTiles) trace[j * kTraceSlots + 7] = clk64();
         uint64_t voff = (uint64_t)((s * G::VBYTES) >> 4);
@@ -401,11 +441,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           voff += ((uint64_t)(lbo >> 4) << 16) - ((uint64_t)(16384u >> 4) << 16);
         }
         // P of keys [64h, 64h + 64) sits at the start of S half h
-        const uint32_t aP = tbase + kColS0 + (j & 1) * 128;
+        const uint32_t aP = tbase + kColS0 + (jg & 1) * 128;
         if (elect_one()) {
           if (DT == 1 && BS)
-            tmem_cp_32x128b_x4(tbase + kColSFA + (j & 1) * 4,
-                               smem_desc(sbase + G::OFF_SF + (j & 1) * 512, 16, 128, SW_NONE));
+            tmem_cp_32x128b_x4(tbase + kColSFA + (jg & 1) * 4,
+                               smem_desc(sbase + G::OFF_SF + (jg & 1) * 512, 16, 128, SW_NONE));
           if (trace && j < kTraceTiles) trace[j * kTraceSlots + 8] = clk64();
 #pragma unroll
           for (int kk = 0; kk < G::PV_STEPS; ++kk) {
@@ -416,7 +456,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else {
               // 32 keys per step = 8 columns of 4 x e4m3; scale byte kk
               // N = d_v + 16: V and the ones block in one instruction
-              const uint32_t sfa = (tbase + kColSFA + (j & 1) * 4) | ((uint32_t)kk << 30);
+              const uint32_t sfa = (tbase + kColSFA + (jg & 1) * 4) | ((uint32_t)kk << 30);
               const uint32_t sfb = (tbase + kColSFB) | ((uint32_t)kk << 30);
               mma_mxf8_ts(tbase + kColO, aP + (kk >> 1) * 64 + (kk & 1) * 8, dvv[kk] + voff,
                           idesc_mx(1u, 128, DV + 16, kk, kk), sfa, sfb, acc);
@@ -430,14 +470,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (trace && lane == 0 && j < kTraceTiles) trace[j * kTraceSlots + 10] = clk64();
         return true;
       };
-      bool ok = wait_all(bar_q, 0);
-      for (int j = 0; ok && j < n_kv; ++j) {
-        if (!issue_qk(j)) { ok = false; break; }
-        if (j > 0 && !issue_pv(j - 1)) { ok = false; break; }
+      int jt = 0, nq = 0;
+      bool ok = true;
+      for (int k = 0, u = unit_at(0); ok && u < n_units; u = PERSIST ? unit_at(++k) : n_units) {
+        const Unit w = unit_of(p, u);
+        if (w.n_kv == 0) continue;
+        trace = traced_unit(w) ? trace_buf : nullptr;
+        if (!wait_all(bar_q, nq & 1)) { ok = false; break; }
+        for (int j = 0; j < w.n_kv; ++j) {
+          if (!issue_qk(jt + j, j)) { ok = false; break; }
+          if (j == w.n_kv - 1) {
+            // the unit's last QK: Q may be replaced once it completes
+            if (elect_one()) tc_commit(bar_qfree);
+            __syncwarp();
+          }
+          if (j == 1 && nq > 0) {
+            // PV_0 overwrites O: the softmax must have read the last unit's
+            if (!wait_all(bar_ofree, (nq - 1) & 1)) { ok = false; break; }
+          }
+          if (j > 0 && !issue_pv(jt + j - 1, j - 1)) { ok = false; break; }
+        }
+        if (!ok) break;
+        if (w.n_kv == 1 && nq > 0 && !wait_all(bar_ofree, (nq - 1) & 1)) { ok = false; break; }
+        if (!issue_pv(jt + w.n_kv - 1, w.n_kv - 1)) { ok = false; break; }
+        if (elect_one()) tc_commit(bar_ofinal);
+        __syncwarp();
+        jt += w.n_kv;
+        ++nq;
       }
-      if (ok && !issue_pv(n_kv - 1)) ok = false;
-      if (ok && elect_one()) tc_commit(bar_ofinal);
-      __syncwarp();
       if (!ok && lane == 0) fail();
     }
   } else {
@@ -453,8 +513,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int half = lane >> 4;
     const int row = qd * 32 + sub * 16 + (lane & 15);  // query row == TMEM lane
     const uint32_t col_h = (uint32_t)half * 64;
-    const int i = q0 + row;
-    const int row_lim = p.causal ? min(i + shift, p.Sk - 1) : p.Sk - 1;
     const uint32_t lane_off = (uint32_t)(qd * 32 + sub * 16) << 16;  // 16-lane group
     constexpr unsigned kFull = 0xffffffffu;
     float c = p.softmax_scale * 1.4426950408889634f;  // log2(e)
@@ -482,11 +540,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     int eref = kInvalidExp;   // FP8: reference exponent E (invalid until a key is seen)
     float l = 0.0f;           // BF16: this thread's half of the row sum (fp32, unrounded p)
     bool ok = true;
+    int jt = 0, nq = 0;       // key tiles and units with work so far (as the MMA warp counts)
 
     // O holds tiles < j at the old reference: rescale this thread's 64 O
     // columns by f once PV_{j-1} has landed (rare: the reference is lazy)
-    auto rescale_o = [&](int j, float f) -> bool {
-      const bool w2 = mbar_wait(bar_kvdone + (j - 1) % G::NS, ((j - 1) / G::NS) & 1, lim, abort_flag);
+    auto rescale_o = [&](int jg, float f) -> bool {
+      const bool w2 = mbar_wait(bar_kvdone + (jg - 1) % G::NS, ((jg - 1) / G::NS) & 1, lim, abort_flag);
       if (!__all_sync(kFull, w2)) return false;
       tc_fence_after();
 #pragma unroll 1
@@ -510,9 +569,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       return true;
     };
 
+    for (int k = 0, u = unit_at(0); ok && u < n_units; u = PERSIST ? unit_at(++k) : n_units) {
+    const Unit wu = unit_of(p, u);
+    const int n_kv = wu.n_kv, min_lim = wu.min_lim, b = wu.b, h = wu.h;
+    const bool traced = traced_unit(wu);
+    uint64_t* const trace = traced ? trace_buf : nullptr;
+    const int i = wu.q0 + row;
+    const int row_lim = p.causal ? min(i + shift, p.Sk - 1) : p.Sk - 1;
+    yref = -INFINITY;
+    eref = kInvalidExp;
+    l = 0.0f;
     for (int j = 0; ok && j < n_kv; ++j) {
-      const int buf = j & 1;
-      const bool w = mbar_wait(bar_sfull + buf, (j >> 1) & 1, lim, abort_flag);
+      const int jg = jt + j;
+      const int buf = jg & 1;
+      const bool w = mbar_wait(bar_sfull + buf, (jg >> 1) & 1, lim, abort_flag);
       if (!__all_sync(kFull, w)) { ok = false; break; }
       tc_fence_after();
       if (trace && warp == 0 && lane == 0 && j < kTraceTiles) trace[j * kTraceSlots + 0] = clk64();
@@ -554,7 +624,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float f = (nref == -INFINITY || yref == nref) ? 1.0f : ex2_approx(yref - nref);
           yref = nref;
           l *= f;
-          if (j > 0 && !rescale_o(j, f)) { ok = false; break; }
+          if (j > 0 && !rescale_o(jg, f)) { ok = false; break; }
         }
         const float nb = yref == -INFINITY ? 0.0f : -yref;
         uint32_t pk[32];
@@ -600,7 +670,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (__builtin_expect(j > 0 && __any_sync(kFull, grow), 0)) {
           // O and the row sum hold tiles < j at scale 2^(-eref): move them
           // to 2^(-nref) exactly
-          if (!rescale_o(j, grow ? pow2i(max(eref - nref, -126)) : 1.0f)) { ok = false; break; }
+          if (!rescale_o(jg, grow ? pow2i(max(eref - nref, -126)) : 1.0f)) { ok = false; break; }
         }
         eref = nref;
         const bool v = e > kInvalidExp;
@@ -666,62 +736,59 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (warp == 5) trace[j * kTraceSlots + 12] = clk64();
       }
     }
-    if (!ok) {
-      if (lane == 0) fail();
-    } else {
+    if (!ok) break;
+    {
       // ------------------------------------------------------------ epilogue
       bool wok = true;
-      if (n_kv > 0) wok = __all_sync(kFull, mbar_wait(bar_ofinal, 0, lim, abort_flag));
+      if (n_kv > 0) wok = __all_sync(kFull, mbar_wait(bar_ofinal, nq & 1, lim, abort_flag));
       if (!wok) {
-        if (lane == 0) fail();
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      // O and the row sum into registers, then hand O back to the MMA warp
+      // (the next unit's first PV overwrites it) before the stores
+      uint32_t o[64];
+      float L = 0.0f, lse_v = -INFINITY;
+      if (n_kv > 0) {
+        tmem_ld16x2_32<64>(tbase + lane_off + kColO, *reinterpret_cast<uint32_t(*)[32]>(o));
+        tmem_ld16x2_32<64>(tbase + lane_off + kColO + 32, *reinterpret_cast<uint32_t(*)[32]>(o + 32));
+        uint32_t rs = 0u;
+        if (DT == 1) tmem_ld16x2_1<1>(tbase + lane_off + kColRS, rs);  // columns RS / RS + 1: equal
+        tmem_ld_wait_regs(*reinterpret_cast<uint32_t(*)[32]>(o), *reinterpret_cast<uint32_t(*)[32]>(o + 32));
+        asm volatile("" : "+r"(rs)::"memory");  // rs, too, is read only after the wait
+        if (DT == 1) L = __uint_as_float(rs);
+        tc_fence_before();
+        mbar_arrive(bar_ofree);
       } else {
-        tc_fence_after();
-        float L, lse_v = -INFINITY;
-        if (DT == 1) {
-          L = 0.0f;
-          if (n_kv > 0) {
-            uint32_t rs;
-            tmem_ld16x2_1<1>(tbase + lane_off + kColRS, rs);  // columns RS / RS + 1: equal
-            tmem_ld_wait();
-            L = __uint_as_float(rs);
-          }
-        } else {
-          L = l + __shfl_xor_sync(kFull, l, 16);  // same value in both halves
-        }
-        // no visible key: L == 0 (FP8), or the reference never left -inf (BF16;
-        // the software exp2 maps masked scores to ~2^-126 instead of 0)
-        const bool empty = !(L > 0.0f) || (DT == 0 && yref == -INFINITY);
-        const float inv = empty ? 0.0f : vscale / L;
-        if (!empty) {
-          const float ref = DT == 0 ? yref : (float)eref;
-          lse_v = (ref + __log2f(L)) * 0.6931471805599453f;
-        }
-        __nv_bfloat16* orow =
-            static_cast<__nv_bfloat16*>(p.out) + (((int64_t)b * p.Sq + i) * p.Hq + h) * DV + col_h;
-#pragma unroll 1
-        for (int ch = 0; ch < 2; ++ch) {
-          uint32_t o[32];
-          if (n_kv > 0) {
-            tmem_ld16x2_32<64>(tbase + lane_off + kColO + ch * 32, o);
-            tmem_ld_wait();
-          } else {
 #pragma unroll
-            for (int q = 0; q < 32; ++q) o[q] = 0u;
-          }
-          uint32_t pk[16];
+        for (int q = 0; q < 64; ++q) o[q] = 0u;
+      }
+      if (DT == 0) L = l + __shfl_xor_sync(kFull, l, 16);  // same value in both halves
+      // no visible key: L == 0 (FP8), or the reference never left -inf (BF16;
+      // the software exp2 maps masked scores to ~2^-126 instead of 0)
+      const bool empty = !(L > 0.0f) || (DT == 0 && yref == -INFINITY);
+      const float inv = empty ? 0.0f : vscale / L;
+      if (!empty) {
+        const float ref = DT == 0 ? yref : (float)eref;
+        lse_v = (ref + __log2f(L)) * 0.6931471805599453f;
+      }
+      if (i < p.Sq) {
+        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) +
+                                              (((int64_t)b * p.Sq + i) * p.Hq + h) * DV + col_h);
 #pragma unroll
-          for (int q = 0; q < 16; ++q)
-            pk[q] = pack_bf16x2(__uint_as_float(o[2 * q]) * inv, __uint_as_float(o[2 * q + 1]) * inv);
-          if (i < p.Sq) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-          }
-        }
-        if (half == 0 && p.lse && i < p.Sq) p.lse[((int64_t)b * p.Hq + h) * p.Sq + i] = lse_v;
+        for (int q = 0; q < 8; ++q)
+          dst[q] = make_uint4(pack_bf16x2(__uint_as_float(o[8 * q]) * inv, __uint_as_float(o[8 * q + 1]) * inv),
+                              pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv, __uint_as_float(o[8 * q + 3]) * inv),
+                              pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv, __uint_as_float(o[8 * q + 5]) * inv),
+                              pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv, __uint_as_float(o[8 * q + 7]) * inv));
+        if (half == 0 && p.lse) p.lse[((int64_t)b * p.Hq + h) * p.Sq + i] = lse_v;
       }
     }
+    jt += n_kv;
+    if (n_kv > 0) ++nq;
+    }  // units
+    if (!ok && lane == 0) fail();
   }
 
   tc_fence_before();
@@ -818,11 +885,29 @@ static cudaError_t launch_variant(const AttnLaunch& a, cudaStream_t st) {
     mQ2 = mQ;
     mK2 = mK;
   }
-  auto kern = p.dbg ? attn_fwd_kernel<DT, DQK, DV, MODE, BS, 1> : attn_fwd_kernel<DT, DQK, DV, MODE, BS, 0>;
+  const long long n_units = (long long)p.n_qtiles * p.B * p.Hq;
+  if (n_units <= 0) return cudaSuccess;
+  if (n_units > 0x7fffffffLL) return cudaErrorInvalidValue;
+  // Short sequences (at most 64 query tiles) run persistent: one CTA per SM
+  // (all of TMEM), each walking its share of the units (see unit_at in the
+  // kernel), so a unit's loads and first QK overlap the previous unit's tail.
+  // Longer ones launch a CTA per unit from a one-unit instantiation: the
+  // hardware scheduler then balances units of very different lengths better
+  // than the static share, and the per-unit setup is a small part of a long
+  // unit.
+  long long nblocks = n_units;
+  const bool persist = p.n_qtiles <= 64;
+  if (persist) {
+    int dev = 0, sms = 0;
+    cudaError_t e0 = cudaGetDevice(&dev);
+    if (e0 == cudaSuccess) e0 = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e0 != cudaSuccess) return e0;
+    if (sms > 0 && sms < nblocks) nblocks = sms;
+  }
+  auto kern = p.dbg ? (persist ? attn_fwd_kernel<DT, DQK, DV, MODE, BS, 1, 1> : attn_fwd_kernel<DT, DQK, DV, MODE, BS, 1, 0>)
+                    : (persist ? attn_fwd_kernel<DT, DQK, DV, MODE, BS, 0, 1> : attn_fwd_kernel<DT, DQK, DV, MODE, BS, 0, 0>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM);
   if (e != cudaSuccess) return e;
-  const long long nblocks = (long long)p.n_qtiles * p.B * p.Hq;
-  if (nblocks <= 0) return cudaSuccess;
   kern<<<(unsigned)nblocks, kThreads, G::SMEM, st>>>(mQ, mQ2, mK, mK2, mV, p);
   return cudaGetLastError();
 }

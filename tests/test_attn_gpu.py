@@ -150,6 +150,16 @@ def test_large_logits_lazy_rescale(dtype):
 
 
 @pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("Sq,Sk,causal", [(600, 600, True), (300, 100, True), (200, 520, False)])
+def test_many_units_per_cta(dtype, Sq, Sk, causal):
+    # Short sequences run persistent CTAs that take several (tile, head)
+    # units each: 2 x 80 heads give far more units than SMs, so every CTA
+    # crosses unit boundaries (barrier phases carried over, O and Q handed
+    # back between units), including units with no visible key (Sq > Sk).
+    check_against_oracle(Case(2, Sq, Sk, 80, 16, 128, 128, dtype=dtype, causal=causal, seed=Sq + Sk))
+
+
+@pytest.mark.parametrize("dtype", DTYPES)
 def test_bitwise_deterministic(dtype):
     c = Case(1, 1000, 1000, 4, 2, 128, 128, dtype=dtype, seed=7)
     o0, l0 = c.run_gpu()
