@@ -21,7 +21,8 @@
 //              a warp, threads t and t+16 share a row, thread t taking keys
 //              0-63 of every tile and thread t+16 keys 64-127 (one 64-key
 //              scale block each; 16x32bx2 TMEM accesses)
-//   warp 8     TMA producer (Q once, then K/V tiles through an NS-stage ring)
+//   warp 8     TMA producer (Q per unit, then K and V tiles through two
+//              NS-stage rings that refill independently)
 //   warp 9     TMEM allocator and tcgen05 issuer (the whole warp runs the
 //              loop, one elected lane issues)
 // Tensor memory (512 columns x 128 lanes, fp32 words):
@@ -82,7 +83,7 @@ struct Geo {
   static constexpr int OFF_SF = OFF_ONES + ONES_BYTES;     // FP8: [2 buf] 512 B scale tiles
   static constexpr int SF_BYTES = DT == 1 ? 1024 : 0;
   static constexpr int OFF_BAR = OFF_SF + SF_BYTES;
-  static constexpr int NBAR = 1 + 2 * NS + 2 + 2 + 1 + 2;
+  static constexpr int NBAR = 1 + 4 * NS + 2 + 2 + 1 + 2;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;  // + alignment slack
   static_assert(SMEM <= 232448, "227 KB of shared memory per CTA");
   static_assert(DV == 128, "the two halves of a row split d_v = 128 in 64 + 64");
@@ -249,14 +250,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + G::OFF_BAR);
   uint64_t* bar_q = bars;
-  uint64_t* bar_kvfull = bars + 1;           // [NS] K_j and V_j landed
-  // bar_kvdone[s] completes when PV_j (j = s mod NS) is done: it frees the
-  // K/V stage and tells the softmax that O holds tiles <= j.  Softmax j
-  // (j >= 1) waits for PV_{j-1}: of that stage's phases only (j-1)/NS - 1
-  // (done long ago) or (j-1)/NS can be complete, since PV_{j-1+NS} needs
+  // With two stages (BF16 at d_qk = 192) K and V have separate rings: K_j is
+  // consumed by QK_j, about two tiles before PV_j needs V_j, so a K stage
+  // frees and refills much earlier, which a two-stage ring needs to hide the
+  // load latency.  With more stages K_j and V_j share a stage: both land on
+  // bar_kfull, and PV_j's commit on bar_vfree frees both (one commit and one
+  // wait fewer per tile for the MMA warp, which measured faster there).
+  constexpr bool kSplit = G::NS == 2;
+  uint64_t* bar_kfull = bars + 1;             // [NS] K_j (and V_j unless split) landed
+  uint64_t* bar_kfree = bar_kfull + G::NS;    // [NS] QK_j done: K stage reusable
+  uint64_t* bar_vfull = bar_kfree + G::NS;    // [NS] V_j landed
+  // bar_vfree[s] completes when PV_j (j = s mod NS) is done: it frees the V
+  // stage and tells the softmax that O holds tiles <= j.  Softmax j
+  // (j >= 1) waits for PV_{j-1}: of that stage's phases only the awaited
+  // one or the one before can be complete, since PV_{j-1+NS} needs
   // P_{j-1+NS}; so the parity test is unambiguous.
-  uint64_t* bar_kvdone = bar_kvfull + G::NS;  // [NS]
-  uint64_t* bar_sfull = bar_kvdone + G::NS;   // [2]
+  uint64_t* bar_vfree = bar_vfull + G::NS;    // [NS]
+  uint64_t* bar_sfull = bar_vfree + G::NS;    // [2]
   uint64_t* bar_pfull = bar_sfull + 2;        // [2]
   uint64_t* bar_ofinal = bar_pfull + 2;       // [1] last PV of a unit landed
   // A CTA runs units one after another (persistent); the barrier phases run
@@ -294,8 +304,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 1);
     for (int s = 0; s < G::NS; ++s) {
-      mbar_init(bar_kvfull + s, 1);
-      mbar_init(bar_kvdone + s, 1);
+      mbar_init(bar_kfull + s, 1);
+      mbar_init(bar_kfree + s, 1);
+      mbar_init(bar_vfull + s, 1);
+      mbar_init(bar_vfree + s, 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar_sfull + s, 1);
@@ -354,23 +366,74 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_4d(sq + c * 16384, narrow ? (const void*)&tmQ2 : (const void*)&tmQ, bar_q,
                       c * 128 / G::ES, w.h, w.q0, w.b);
         }
-        for (int j = 0; j < w.n_kv; ++j, ++jt) {
-          const int s = jt % G::NS;
-          const uint32_t ph = ((jt / G::NS) & 1) ^ 1;  // first pass through the ring: free
-          if (!mbar_wait(bar_kvdone + s, ph, lim, abort_flag)) { ok = false; break; }
-          uint8_t* sk = smem + G::OFF_K + s * G::KBYTES;
-          uint8_t* sv = smem + G::OFF_V + s * G::VBYTES;
-          mbar_arrive_expect_tx(bar_kvfull + s, G::KBYTES + G::VBYTES);
+        if constexpr (!kSplit) {
+          for (int j = 0; j < w.n_kv; ++j) {
+            const int x = jt + j, s = x % G::NS;
+            // the stage is free once PV of its previous tile is done (first pass: free)
+            if (!mbar_wait(bar_vfree + s, ((x / G::NS) & 1) ^ 1, lim, abort_flag)) { ok = false; break; }
+            uint8_t* sk = smem + G::OFF_K + s * G::KBYTES;
+            uint8_t* sv = smem + G::OFF_V + s * G::VBYTES;
+            mbar_arrive_expect_tx(bar_kfull + s, G::KBYTES + G::VBYTES);
 #pragma unroll
-          for (int c = 0; c < G::NCH; ++c) {
-            const bool narrow = (c == G::NCH - 1) && G::LASTW == 64;
-            tma_load_4d(sk + c * 16384, narrow ? (const void*)&tmK2 : (const void*)&tmK,
-                        bar_kvfull + s, c * 128 / G::ES, w.g, j * kTile, w.b);
+            for (int c = 0; c < G::NCH; ++c) {
+              const bool narrow = (c == G::NCH - 1) && G::LASTW == 64;
+              tma_load_4d(sk + c * 16384, narrow ? (const void*)&tmK2 : (const void*)&tmK,
+                          bar_kfull + s, c * 128 / G::ES, w.g, j * kTile, w.b);
+            }
+#pragma unroll
+            for (int c = 0; c < G::VCH; ++c)
+              tma_load_4d(sv + c * 16384, &tmV, bar_kfull + s, c * 128 / G::ES, w.g, j * kTile, w.b);
           }
+        } else {
+          // K runs ahead of V inside the unit; each ring refills as its stages free
+          int jk = 0, jv = 0;
+          uint64_t t0 = 0;
+          uint32_t idle = 0;
+          while (jv < w.n_kv) {
+            bool progressed = false;
+            if (jk < w.n_kv) {
+              const int x = jt + jk, s = x % G::NS;
+              if (mbar_test_wait(smem_u32(bar_kfree + s), ((x / G::NS) & 1) ^ 1)) {  // first pass: free
+                uint8_t* sk = smem + G::OFF_K + s * G::KBYTES;
+                mbar_arrive_expect_tx(bar_kfull + s, G::KBYTES);
 #pragma unroll
-          for (int c = 0; c < G::VCH; ++c)
-            tma_load_4d(sv + c * 16384, &tmV, bar_kvfull + s, c * 128 / G::ES, w.g, j * kTile, w.b);
+                for (int c = 0; c < G::NCH; ++c) {
+                  const bool narrow = (c == G::NCH - 1) && G::LASTW == 64;
+                  tma_load_4d(sk + c * 16384, narrow ? (const void*)&tmK2 : (const void*)&tmK,
+                              bar_kfull + s, c * 128 / G::ES, w.g, jk * kTile, w.b);
+                }
+                ++jk;
+                progressed = true;
+              }
+            }
+            if (jv < jk) {
+              const int x = jt + jv, s = x % G::NS;
+              if (mbar_test_wait(smem_u32(bar_vfree + s), ((x / G::NS) & 1) ^ 1)) {
+                uint8_t* sv = smem + G::OFF_V + s * G::VBYTES;
+                mbar_arrive_expect_tx(bar_vfull + s, G::VBYTES);
+#pragma unroll
+                for (int c = 0; c < G::VCH; ++c)
+                  tma_load_4d(sv + c * 16384, &tmV, bar_vfull + s, c * 128 / G::ES, w.g, jv * kTile, w.b);
+                ++jv;
+                progressed = true;
+              }
+            }
+            if (progressed) {
+              idle = 0;
+            } else {
+              // nothing to load yet: back off; give up after the time limit
+              if (idle == 0) t0 = globaltimer_ns();
+              ++idle;
+              __nanosleep(32);
+              if ((idle & 63u) == 0 && (*abort_flag || globaltimer_ns() - t0 > lim)) {
+                ok = false;
+                break;
+              }
+            }
+          }
         }
+        if (!ok) break;
+        jt += w.n_kv;
         ++nq;
       }
       if (!ok) fail();
@@ -410,7 +473,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint64_t* trace = nullptr;
       auto issue_qk = [&](int jg, int j) -> bool {
         const int s = jg % G::NS;
-        if (!wait_all(bar_kvfull + s, (jg / G::NS) & 1)) return false;
+        if (!wait_all(bar_kfull + s, (jg / G::NS) & 1)) return false;
         tc_fence_after();
         if (trace && lane == 0 && j < kTraceTiles) trace[j * kTraceSlots + 5] = clk64();
         const uint32_t dS = tbase + kColS0 + (jg & 1) * 128;
@@ -424,6 +487,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               mma_f8_ss(dS, dq[kk], dk[kk] + koff, idesc_qk, kk > 0);
             if (trace && kk == 1 && j < kTraceTiles) trace[j * kTraceSlots + 13] = clk64();
           }
+          if (kSplit) tc_commit(bar_kfree + s);
           tc_commit(bar_sfull + (jg & 1));
         }
         __syncwarp();
@@ -433,6 +497,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto issue_pv = [&](int jg, int j) -> bool {
         const int s = jg % G::NS;
         if (!wait_all(bar_pfull + (jg & 1), (jg >> 1) & 1)) return false;
+        if (kSplit && !wait_all(bar_vfull + s, (jg / G::NS) & 1)) return false;
         tc_fence_after();
         if (trace && lane == 0 && j < kTraceTiles) trace[j * kTraceSlots + 7] = clk64();
         uint64_t voff = (uint64_t)((s * G::VBYTES) >> 4);
@@ -464,7 +529,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (trace && kk == 1 && j < kTraceTiles) trace[j * kTraceSlots + 14] = clk64();
           }
           if (trace && j < kTraceTiles) trace[j * kTraceSlots + 9] = clk64();
-          tc_commit(bar_kvdone + s);
+          tc_commit(bar_vfree + s);
         }
         __syncwarp();
         if (trace && lane == 0 && j < kTraceTiles) trace[j * kTraceSlots + 10] = clk64();
@@ -545,7 +610,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // O holds tiles < j at the old reference: rescale this thread's 64 O
     // columns by f once PV_{j-1} has landed (rare: the reference is lazy)
     auto rescale_o = [&](int jg, float f) -> bool {
-      const bool w2 = mbar_wait(bar_kvdone + (jg - 1) % G::NS, ((jg - 1) / G::NS) & 1, lim, abort_flag);
+      const bool w2 = mbar_wait(bar_vfree + (jg - 1) % G::NS, ((jg - 1) / G::NS) & 1, lim, abort_flag);
       if (!__all_sync(kFull, w2)) return false;
       tc_fence_after();
 #pragma unroll 1
