@@ -52,6 +52,8 @@ def parse():
     ap.add_argument("--S", type=int, default=None)
     ap.add_argument("--dtype", default="leanp", choices=["leanp", "exact", "bf16"])
     ap.add_argument("--hadamard", action="store_true")
+    ap.add_argument("--T", type=int, default=8, help="FP8 headroom T (block maximum lands in (2^(T-1), 2^T])")
+    ap.add_argument("--no-energy", action="store_true", help="skip the attention-only power measurement")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-e2e", action="store_true")
@@ -150,10 +152,12 @@ class ClockSampler:
                 if val.lower().startswith("active"):
                     reasons.add(nm)
         loaded = [s for s, p in zip(sm, power) if p > 300] or sm
+        loaded_p = [p for p in power if p > 300] or power
         return {"sm_mhz": statistics.median(loaded) if loaded else None,
                 "sm_max_mhz": max(smax) if smax else None,
                 "reasons": sorted(reasons), "samples": len(sm),
-                "power_w_max": max(power) if power else None}
+                "power_w_max": max(power) if power else None,
+                "power_w_mean": statistics.mean(loaded_p) if loaded_p else None}
 
 
 def measured_peaks():
@@ -188,7 +192,7 @@ def load_traffic(key: str):
 class Step:
     """The hot path for one workload on one GPU; inputs resident in HBM."""
 
-    def __init__(self, w: workloads.Workload, dtype: str, hadamard: bool, seed_offset: int = 0):
+    def __init__(self, w: workloads.Workload, dtype: str, hadamard: bool, seed_offset: int = 0, T: int = 8):
         import bf16_causal_prefill_02_b200 as zq
 
         self.zq, self.w, self.dtype, self.hadamard = zq, w, dtype, hadamard
@@ -210,6 +214,7 @@ class Step:
             self.ds = torch.zeros(3, dtype=torch.float32, device=dev)
             self.ws = torch.empty(3, zq.zq_quantize_workspace_bytes(), dtype=torch.uint8, device=dev)
         self.mode = zq.ZQ_SOFTMAX_EXACT if dtype == "exact" else zq.ZQ_SOFTMAX_LEANP
+        self.T = T
         self.ev = []
 
     def launches_per_step(self) -> int:
@@ -224,7 +229,7 @@ class Step:
         else:
             zq.attn_fwd(self.qc, self.kc, self.vc, out=self.out, lse=self.lse,
                         q_descale=self.ds[0:1], k_descale=self.ds[1:2], v_descale=self.ds[2:3],
-                        softmax_mode=self.mode, block_scale=True, headroom_T=8)
+                        softmax_mode=self.mode, block_scale=True, headroom_T=self.T)
         if ev is not None:
             ev[1].record()
 
@@ -353,7 +358,7 @@ def oracle_steps(w, dtype, steps, warmup, rows_per_step, hadamard=False):
 def run_ours(args, rank, world, w):
     import bf16_causal_prefill_02_b200 as zq  # noqa: F401  (fails loudly without the .so)
 
-    step = Step(w, args.dtype, args.hadamard, seed_offset=rank)
+    step = Step(w, args.dtype, args.hadamard, seed_offset=rank, T=args.T)
     flops = w.causal_flops()
     sampler = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
     # warm-up + attention-only event timing for the roofline
@@ -380,6 +385,31 @@ def run_ours(args, rank, world, w):
     ms_step = ms_total / args.steps
     total_flops = sum_over_ranks(flops, world)
     value = total_flops / (ms_step * 1e-3) / 1e12
+    # energy: attention launches back to back for about a second while
+    # nvidia-smi samples the board power every 100 ms
+    energy = None
+    if not args.no_energy:
+        n = max(1, int(1000.0 / max(attn_ms, 1e-3)))
+        es = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
+        es.start()
+        time.sleep(0.3)
+        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        step.attention()
+        b0.record(st)
+        for _ in range(n):
+            step.attention()
+        b1.record(st)
+        torch.cuda.synchronize()
+        ec = es.stop()
+        e_ms = b0.elapsed_time(b1) / n
+        pw = ec.get("power_w_mean")
+        if pw:
+            tf = flops / (e_ms * 1e-3) / 1e12
+            energy = {"tflop_per_joule": round(tf / pw, 3), "attn_tflops": round(tf, 1),
+                      "power_w_mean": round(pw, 1), "sm_mhz": ec.get("sm_mhz"),
+                      "reasons": ec.get("reasons"), "samples": ec.get("samples"),
+                      "basis": "%d back-to-back attention launches; board power.draw from nvidia-smi "
+                               "every 100 ms, mean over the loaded samples" % n}
     # end to end from host buffers
     e2e = None
     if not args.no_e2e:
@@ -402,7 +432,7 @@ def run_ours(args, rank, world, w):
         "config": {"workload": "%s_%s%s" % (w.name, args.dtype, "_hadamard" if args.hadamard else ""),
                    "B": w.B, "S": w.S, "Hq": w.Hq, "Hkv": w.Hkv, "d_qk": w.dqk, "d_v": w.dv,
                    "causal": True, "softmax": args.dtype,
-                   "block_scale": kind == "fp8", "headroom_T": 8 if kind == "fp8" else None,
+                   "block_scale": kind == "fp8", "headroom_T": args.T if kind == "fp8" else None,
                    "step": ("quantise Q,K,V (fp32->e4m3) + attention" if kind == "fp8" else "attention"),
                    "l2": "inputs larger than L2 (%.0f MB fp32 Q/K/V), no flush" %
                          (3 * w.B * w.S * w.Hq * w.dqk * 4 / 1e6),
@@ -413,6 +443,7 @@ def run_ours(args, rank, world, w):
                      "frac_of_datasheet_dense": round(achieved / DATASHEET_DENSE_TFLOPS[kind], 4),
                      "attn_ms": round(attn_ms, 4)},
         "clocks": clocks,
+        "energy": energy,
         "e2e": e2e,
         "gpu_launches": step.launches_per_step() * args.steps,
     }
@@ -464,7 +495,8 @@ def main():
             print(json.dumps({"sweep": r["config"]["workload"], "S": r["config"]["S"],
                               "value": r["value"], "attn_tflops": r["roofline"]["achieved"],
                               "frac": r["roofline"]["frac"], "ms_per_step": r["ms_per_step"],
-                              "attn_ms": r["roofline"]["attn_ms"], "clocks": r["clocks"]}), flush=True)
+                              "attn_ms": r["roofline"]["attn_ms"], "clocks": r["clocks"],
+                              "energy": r["energy"]}), flush=True)
     if world > 1:
         import torch.distributed as dist
 
