@@ -63,6 +63,7 @@ def _L():
         lib.zo_e4m3_encode_rne_sat.argtypes = [f64]
         lib.zo_e4m3_encode_rne_sat.restype = ctypes.c_uint8
         lib.zo_fwht128_f32.argtypes = [P]
+        lib.zo_fwht64_f32.argtypes = [P]
         lib.zo_quantize_fp8.argtypes = [P, i32, i64, i32, i32, P, P]
         lib.zo_quantize_fp8.restype = i32
         lib.zo_attn_ref.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, i32, f64, i32, P, i64, P, P]
@@ -117,6 +118,19 @@ def fwht128(x: np.ndarray) -> np.ndarray:
     for r in range(flat.shape[0]):
         row = np.ascontiguousarray(flat[r])
         lib.zo_fwht128_f32(_ptr(row))
+        flat[r] = row
+    return flat.reshape(x.shape)
+
+
+def fwht64(x: np.ndarray) -> np.ndarray:
+    """Unnormalised 64-point FWHT of each 64-slice, fp32 butterflies."""
+    x = np.array(x, dtype=np.float32, copy=True, order="C")
+    assert x.shape[-1] % 64 == 0
+    flat = x.reshape(-1, 64)
+    lib = _L()
+    for r in range(flat.shape[0]):
+        row = np.ascontiguousarray(flat[r])
+        lib.zo_fwht64_f32(_ptr(row))
         flat[r] = row
     return flat.reshape(x.shape)
 

@@ -24,6 +24,8 @@
  *   zo_fwht128_f32      unnormalised 128-point Walsh-Hadamard transform in
  *        fp32, butterflies at strides 1,2,...,64.  [P2 "Perche l'FP8 non
  *        basta da solo": Hadamard rotation of Q and K]
+ *   zo_fwht64_f32       the same for 64 points (strides 1..32); the d = 192
+ *        rotation uses it, scaled by fl32(sqrt 2), on channels 128..191.
  *   zo_quantize_fp8     per-tensor amax quantiser (R3).
  *   zo_attn_ref         exact fp64 softmax(QK^T*scale + causal mask)V (R1).
  *   zo_attn_fp8_emul    scalar emulation of the FP8 P path: per-(row,64-key
@@ -107,6 +109,35 @@ void zo_fwht128_f32(float* x) {
       }
 }
 
+/* In-place unnormalised FWHT of 64 fp32 values, as above with h < 64. */
+void zo_fwht64_f32(float* x) {
+  for (int h = 1; h < 64; h <<= 1)
+    for (int i = 0; i < 64; i += 2 * h)
+      for (int j = i; j < i + h; ++j) {
+        float a = x[j], b = x[j + h];
+        x[j] = a + b;
+        x[j + h] = a - b;
+      }
+}
+
+/* The rotation of one d-channel vector: H128 on every 128-channel slice;
+ * for d = 192 (the MLA query/key width) the last 64 channels get
+ * sqrt(2) * H64 instead, each value multiplied by fl32(sqrt 2) after the
+ * butterflies.  Then (R q).(R k) = 128 q.k for every slice (up to the fp32
+ * rounding of sqrt 2), so one descale factor 2^-3.5 per tensor undoes the
+ * rotation in QK^T for d = 128 and d = 192 alike. */
+static void rotate_vec(float* x, int d) {
+  int c = 0;
+  for (; c + 128 <= d; c += 128) zo_fwht128_f32(x + c);
+  if (c < d) {
+    zo_fwht64_f32(x + c);
+    for (int j = 0; j < 64; ++j) {
+      volatile float y = x[c + j] * 1.41421356237309504880f; /* fl32(sqrt 2), one rounding */
+      x[c + j] = y;
+    }
+  }
+}
+
 static float bf16_bits_to_f32(uint16_t h) {
   uint32_t u = (uint32_t)h << 16;
   float f;
@@ -115,8 +146,8 @@ static float bf16_bits_to_f32(uint16_t h) {
 }
 
 /* Per-tensor FP8 quantiser.  x has n_vec vectors of d channels, fp32
- * (x_dtype 0) or bf16 bits (x_dtype 1).  With hadamard != 0 (d % 128 == 0)
- * every 128-channel slice is rotated first.
+ * (x_dtype 0) or bf16 bits (x_dtype 1).  With hadamard != 0 (d % 128 == 0,
+ * or d == 192) every vector is rotated first (rotate_vec).
  *   amax    = max |x|                       (exact)
  *   inv     = fl32(448 / amax)
  *   q       = e4m3_rne_sat(fl32(x * inv))
@@ -125,7 +156,7 @@ static float bf16_bits_to_f32(uint16_t h) {
  * Returns 0, or -1 for an unsupported argument. */
 int zo_quantize_fp8(const void* x, int x_dtype, int64_t n_vec, int d, int hadamard,
                     uint8_t* out, float* descale) {
-  if (n_vec < 0 || d <= 0 || (hadamard && d % 128)) return -1;
+  if (n_vec < 0 || d <= 0 || (hadamard && d % 128 && d != 192)) return -1;
   int64_t n = n_vec * (int64_t)d;
   float* t = (float*)malloc(sizeof(float) * (size_t)(n > 0 ? n : 1));
   if (!t) return -1;
@@ -134,7 +165,7 @@ int zo_quantize_fp8(const void* x, int x_dtype, int64_t n_vec, int d, int hadama
     t[i] = x_dtype == 0 ? ((const float*)x)[i] : bf16_bits_to_f32(((const uint16_t*)x)[i]);
   if (hadamard) {
 #pragma omp parallel for
-    for (int64_t i = 0; i < n; i += 128) zo_fwht128_f32(t + i);
+    for (int64_t v = 0; v < n_vec; ++v) rotate_vec(t + v * d, d);
   }
   float amax = 0.0f;
 #pragma omp parallel for reduction(max : amax)

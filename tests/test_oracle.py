@@ -121,6 +121,46 @@ def test_quantize_matches_torch_cast(hadamard, src):
     assert np.all(np.abs(deq[big] - x32[big]) <= np.abs(x32[big]) / 16 * 1.0001 + 1e-12)
 
 
+def test_fwht64_matches_scipy_hadamard():
+    rng = np.random.default_rng(12)
+    x = rng.standard_normal((9, 64)).astype(np.float32)
+    H = scipy.linalg.hadamard(64).astype(np.float64)
+    assert np.allclose(oracle.fwht64(x).astype(np.float64), x.astype(np.float64) @ H.T, rtol=0, atol=1e-4)
+    twice = oracle.fwht64(oracle.fwht64(x)).astype(np.float64)
+    assert np.allclose(twice, 64.0 * x, rtol=0, atol=1e-3)
+
+
+@pytest.mark.parametrize("j", [0, 5, 127, 128, 150, 191])
+def test_d192_rotation_one_hot_columns(j):
+    # x = e_j rotates to column j of blockdiag(H128, sqrt2 * H64): every
+    # rotated value has the same magnitude (1, or sqrt 2 in the 64-slice),
+    # so all of them quantise to +-448 with the column's sign pattern.
+    x = np.zeros((1, 192), dtype=np.float32)
+    x[0, j] = 1.0
+    codes, ds = oracle.quantize_fp8(x, hadamard=True)
+    R = np.zeros((192, 192))
+    R[:128, :128] = scipy.linalg.hadamard(128)
+    R[128:, 128:] = np.sqrt(2.0) * scipy.linalg.hadamard(64)
+    col = R[:, j]
+    nz = col != 0
+    assert np.all(codes[0, ~nz] == 0)
+    assert np.all(codes[0, nz & (col > 0)] == 0x7E) and np.all(codes[0, nz & (col < 0)] == 0xFE)
+    amax = np.float32(1.0) if j < 128 else np.float32(np.sqrt(np.float32(2.0)) * np.float32(1.0))
+    assert ds == np.float32(np.float32(amax / np.float32(448.0)) * np.float32(2.0 ** -3.5))
+
+
+def test_d192_rotation_preserves_scores():
+    # (R q).(R k) = 128 q.k for R = blockdiag(H128, sqrt2 H64); through the
+    # quantiser the descale undoes it, up to e4m3 rounding
+    q, k, _ = workloads.make_custom(1, 64, 64, 1, 1, 192, 128, seed=13)
+    q32, k32 = q[0, :, 0].numpy(), k[0, :, 0].numpy()
+    cq, dq = oracle.quantize_fp8(q32, hadamard=True)
+    ck, dk = oracle.quantize_fp8(k32, hadamard=True)
+    s = oracle.dequant_e4m3(cq, float(dq)) @ oracle.dequant_e4m3(ck, float(dk)).T
+    ref = q32.astype(np.float64) @ k32.astype(np.float64).T
+    assert np.sqrt(np.mean((s - ref) ** 2) / np.mean(ref ** 2)) < 0.05
+
+
 def test_quantize_zero_tensor():
     codes, ds = oracle.quantize_fp8(np.zeros((4, 128), dtype=np.float32))
     assert not codes.any() and ds == 0.0
