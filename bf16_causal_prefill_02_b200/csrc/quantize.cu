@@ -109,6 +109,99 @@ __global__ void __launch_bounds__(256) quant_write_kernel(const void* __restrict
   }
 }
 
+// ---------------------------------------------------------------------------
+// d = 192 with rotation (MLA queries and keys): one warp per 192-channel
+// vector.  Lane l holds channels 4l..4l+3 of the 128-slice (rotated by
+// fwht128_warp) and channels 128+2l, 128+2l+1 of the 64-slice, rotated by
+// H64 (stride 1 inside the thread, strides 2..32 through shuffles) and then
+// multiplied by fl32(sqrt 2), so that both slices scale scores by 128.
+template <bool BF16IN>
+__device__ __forceinline__ void load2(const void* x, int64_t i, float (&v)[2]) {
+  if constexpr (BF16IN) {
+    const uint32_t u = *reinterpret_cast<const uint32_t*>(static_cast<const uint16_t*>(x) + i);
+    v[0] = __uint_as_float(u << 16);
+    v[1] = __uint_as_float(u & 0xFFFF0000u);
+  } else {
+    const float2 f = __ldg(reinterpret_cast<const float2*>(static_cast<const float*>(x) + i));
+    v[0] = f.x;
+    v[1] = f.y;
+  }
+}
+
+__device__ __forceinline__ void fwht64x2_warp_scaled(float (&v)[2], int lane) {
+  float a = v[0], b = v[1];
+  v[0] = a + b;  // stride 1
+  v[1] = a - b;
+#pragma unroll
+  for (int m = 1; m <= 16; m <<= 1) {  // strides 2, 4, 8, 16, 32
+    const bool upper = (lane & m) != 0;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      float o = __shfl_xor_sync(0xffffffffu, v[i], m);
+      v[i] = upper ? (o - v[i]) : (v[i] + o);
+    }
+  }
+  v[0] = __fmul_rn(v[0], 1.41421356237309504880f);  // fl32(sqrt 2)
+  v[1] = __fmul_rn(v[1], 1.41421356237309504880f);
+}
+
+template <bool BF16IN>
+__global__ void __launch_bounds__(256) quant192_amax_kernel(const void* __restrict__ x, int64_t n_vec,
+                                                            unsigned* __restrict__ amax_bits) {
+  const int lane = threadIdx.x & 31;
+  const int64_t wstride = (int64_t)gridDim.x * (blockDim.x >> 5);
+  float m = 0.0f;
+  for (int64_t vec = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); vec < n_vec;
+       vec += wstride) {
+    float a[4], c[2];
+    load4<BF16IN>(x, vec * 192 + 4 * lane, a);
+    load2<BF16IN>(x, vec * 192 + 128 + 2 * lane, c);
+    fwht128_warp(a, lane);
+    fwht64x2_warp_scaled(c, lane);
+    m = fmaxf(m, fmaxf(fmaxf(fabsf(a[0]), fabsf(a[1])), fmaxf(fabsf(a[2]), fabsf(a[3]))));
+    m = fmaxf(m, fmaxf(fabsf(c[0]), fabsf(c[1])));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  __shared__ float red[8];
+  if (lane == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float r = red[0];
+    for (int w = 1; w < (int)(blockDim.x >> 5); ++w) r = fmaxf(r, red[w]);
+    atomicMax(amax_bits, __float_as_uint(r));
+  }
+}
+
+template <bool BF16IN>
+__global__ void __launch_bounds__(256) quant192_write_kernel(const void* __restrict__ x, int64_t n_vec,
+                                                             const unsigned* __restrict__ amax_bits,
+                                                             uint8_t* __restrict__ out,
+                                                             float* __restrict__ descale) {
+  const int lane = threadIdx.x & 31;
+  const float amax = __uint_as_float(*amax_bits);
+  const float inv = amax > 0.0f ? __fdiv_rn(448.0f, amax) : 1.0f;
+  if (blockIdx.x == 0 && threadIdx.x == 0)
+    *descale = __fmul_rn(__fdiv_rn(amax, 448.0f), 0.08838834764831845f);  // x fl32(2^-3.5)
+  const int64_t wstride = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t vec = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); vec < n_vec;
+       vec += wstride) {
+    float a[4], c[2];
+    load4<BF16IN>(x, vec * 192 + 4 * lane, a);
+    load2<BF16IN>(x, vec * 192 + 128 + 2 * lane, c);
+    fwht128_warp(a, lane);
+    fwht64x2_warp_scaled(c, lane);
+    const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(
+        make_float2(__fmul_rn(a[0], inv), __fmul_rn(a[1], inv)), __NV_SATFINITE, __NV_E4M3);
+    const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(
+        make_float2(__fmul_rn(a[2], inv), __fmul_rn(a[3], inv)), __NV_SATFINITE, __NV_E4M3);
+    *reinterpret_cast<uint32_t*>(out + vec * 192 + 4 * lane) = (uint32_t)lo | ((uint32_t)hi << 16);
+    const __nv_fp8x2_storage_t t = __nv_cvt_float2_to_fp8x2(
+        make_float2(__fmul_rn(c[0], inv), __fmul_rn(c[1], inv)), __NV_SATFINITE, __NV_E4M3);
+    *reinterpret_cast<uint16_t*>(out + vec * 192 + 128 + 2 * lane) = (uint16_t)t;
+  }
+}
+
 // Host-side launcher; arguments were validated by the caller.
 cudaError_t launch_quantize(const void* x, int x_bf16, int64_t n, int hadamard, void* out,
                             float* descale, void* workspace, cudaStream_t st, int num_sms) {
@@ -116,8 +209,21 @@ cudaError_t launch_quantize(const void* x, int x_bf16, int64_t n, int hadamard, 
   cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(unsigned), st);
   if (e != cudaSuccess) return e;
   const int threads = 256;
-  int64_t want = (n / 4 + threads - 1) / threads;
   int64_t cap = (int64_t)num_sms * 8;
+  if (hadamard == 2) {  // d = 192: one warp per vector
+    const int64_t n_vec = n / 192;
+    int64_t want = (n_vec + (threads / 32) - 1) / (threads / 32);
+    int blocks = (int)(want < cap ? (want > 0 ? want : 1) : cap);
+    if (x_bf16) {
+      quant192_amax_kernel<true><<<blocks, threads, 0, st>>>(x, n_vec, amax);
+      quant192_write_kernel<true><<<blocks, threads, 0, st>>>(x, n_vec, amax, (uint8_t*)out, descale);
+    } else {
+      quant192_amax_kernel<false><<<blocks, threads, 0, st>>>(x, n_vec, amax);
+      quant192_write_kernel<false><<<blocks, threads, 0, st>>>(x, n_vec, amax, (uint8_t*)out, descale);
+    }
+    return cudaGetLastError();
+  }
+  int64_t want = (n / 4 + threads - 1) / threads;
   int blocks = (int)(want < cap ? (want > 0 ? want : 1) : cap);
 #define ZQ_QUANT_LAUNCH(BF, HD)                                                               \
   do {                                                                                        \

@@ -184,14 +184,14 @@ int zq_quantize_fp8(const void* x, int x_dtype, int64_t n_vec, int d, int hadama
   if (n_vec < 0 || d <= 0) return ZQ_ERR_SHAPE;
   if (n_vec > 0 && (!x || !x_fp8)) return ZQ_ERR_NULL;
   if (x_dtype != ZQ_X_F32 && x_dtype != ZQ_X_BF16) return ZQ_ERR_UNSUPPORTED;
-  if (d % 8 != 0 || (hadamard && d % 128 != 0)) return ZQ_ERR_UNSUPPORTED;
+  if (d % 8 != 0 || (hadamard && d % 128 != 0 && d != 192)) return ZQ_ERR_UNSUPPORTED;
   if (n_vec > (int64_t)1 << 40 || n_vec * (int64_t)d > ((int64_t)1 << 40)) return ZQ_ERR_SHAPE;
   if (!aligned16(x) || !aligned16(x_fp8) || !aligned16(workspace)) return ZQ_ERR_ALIGN;
   int sms = 0;
   int rc = check_device(&sms);
   if (rc != ZQ_OK) return rc;
   cudaError_t e = zq::launch_quantize(x, x_dtype == ZQ_X_BF16, n_vec * (int64_t)d,
-                                      hadamard ? 1 : 0, x_fp8, descale, workspace,
+                                      hadamard ? (d % 128 == 0 ? 1 : 2) : 0, x_fp8, descale, workspace,
                                       static_cast<cudaStream_t>(stream), sms);
   return e == cudaSuccess ? ZQ_OK : ZQ_ERR_CUDA;
 }
@@ -202,7 +202,7 @@ int zq_quantize_fp8_noalloc(const void* x, int x_dtype, int64_t n_vec, int d, in
   if (n_vec < 0 || d <= 0) return ZQ_ERR_SHAPE;
   if (n_vec > 0 && (!x || !x_fp8)) return ZQ_ERR_NULL;
   if (x_dtype != ZQ_X_F32 && x_dtype != ZQ_X_BF16) return ZQ_ERR_UNSUPPORTED;
-  if (d % 8 != 0 || (hadamard && d % 128 != 0)) return ZQ_ERR_UNSUPPORTED;
+  if (d % 8 != 0 || (hadamard && d % 128 != 0 && d != 192)) return ZQ_ERR_UNSUPPORTED;
   if (n_vec > (int64_t)1 << 40 || n_vec * (int64_t)d > ((int64_t)1 << 40)) return ZQ_ERR_SHAPE;
   // the scratch this call needs must fit the fixed device array
   if (zq_quantize_workspace_bytes() > zq::noalloc_scratch_capacity()) return ZQ_ERR_SHAPE;
@@ -215,7 +215,7 @@ int zq_quantize_fp8_noalloc(const void* x, int x_dtype, int64_t n_vec, int d, in
   void* scratch = zq::noalloc_scratch_for_device(dev);
   if (!scratch) return ZQ_ERR_CUDA;
   cudaError_t e = zq::launch_quantize(x, x_dtype == ZQ_X_BF16, n_vec * (int64_t)d,
-                                      hadamard ? 1 : 0, x_fp8, descale, scratch,
+                                      hadamard ? (d % 128 == 0 ? 1 : 2) : 0, x_fp8, descale, scratch,
                                       static_cast<cudaStream_t>(stream), sms);
   return e == cudaSuccess ? ZQ_OK : ZQ_ERR_CUDA;
 }

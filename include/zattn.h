@@ -154,7 +154,10 @@ ZQ_API int zq_attn_fwd_debug(const zq_attn_args* args, void* dbg, int dbg_bh, in
  *   x        n_vec vectors of d channels, fp32 (x_dtype ZQ_X_F32) or bf16
  *   hadamard != 0: every 128-channel slice is replaced by H_128 x (Sylvester
  *            order, entries +-1, fp32 butterflies at strides 1,2,...,64);
- *            requires d % 128 == 0.
+ *            requires d % 128 == 0, or d == 192 (the MLA query/key width):
+ *            then channels 128..191 are replaced by sqrt(2) H_64 x (fp32
+ *            butterflies at strides 1..32, then each value times
+ *            fl32(sqrt 2)), which scales scores by 128 like H_128.
  *   amax     = max |x| (after rotation);  inv = fl32(448 / amax)
  *   x_fp8    (n_vec, d) e4m3 bytes = e4m3_rne_satfinite(fl32(x * inv))
  *   descale  one fp32 = fl32(amax / 448), times fl32(2^-3.5) when rotated,
@@ -165,7 +168,7 @@ ZQ_API int zq_attn_fwd_debug(const zq_attn_args* args, void* dbg, int dbg_bh, in
  *            used by another call that runs at the same time.
  * n_vec == 0 writes only the descale (0); x and x_fp8 may then be NULL.
  * Errors: ZQ_ERR_NULL, ZQ_ERR_SHAPE (n_vec < 0, d <= 0), ZQ_ERR_UNSUPPORTED
- *   (x_dtype, hadamard with d % 128 != 0, d % 8 != 0), ZQ_ERR_ALIGN (x,
+ *   (x_dtype, hadamard with d % 128 != 0 and d != 192, d % 8 != 0), ZQ_ERR_ALIGN (x,
  *   x_fp8, workspace not 16-byte aligned), ZQ_ERR_ARCH, ZQ_ERR_CUDA.
  */
 ZQ_API int zq_quantize_fp8(const void* x, int x_dtype, int64_t n_vec, int d, int hadamard,

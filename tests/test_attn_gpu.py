@@ -140,6 +140,15 @@ def test_fp8_hadamard_rotated_inputs(dtype):
     check_against_oracle(c)
 
 
+@pytest.mark.parametrize("dtype", ["exact", "leanp"])
+def test_fp8_hadamard_mla_192(dtype):
+    # d_qk = 192 rotated by H128 (+) sqrt2 * H64 on the CPU quantiser; the
+    # kernel computes attention of the rotated, quantised Q and K
+    q, k, v = workloads.make_custom(1, 400, 400, 2, 2, 192, 128, seed=17)
+    q[..., [7, 140, 181]] *= 20.0
+    check_against_oracle(Case(1, 400, 400, 2, 2, 192, 128, dtype=dtype, hadamard=True, inputs=(q, k, v)))
+
+
 @pytest.mark.parametrize("dtype", ["bf16", "leanp"])
 def test_large_logits_lazy_rescale(dtype):
     # scores growing along the sequence force the reference max / exponent

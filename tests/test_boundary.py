@@ -88,7 +88,7 @@ def test_attn_plain_entry_validates_too():
     ((A, 0, 4, 0, 0, A, A, A), zq.ZQ_ERR_SHAPE),
     ((A, 2, 4, 128, 0, A, A, A), zq.ZQ_ERR_UNSUPPORTED),
     ((A, 0, 4, 12, 0, A, A, A), zq.ZQ_ERR_UNSUPPORTED),
-    ((A, 0, 4, 192, 1, A, A, A), zq.ZQ_ERR_UNSUPPORTED),
+    ((A, 0, 4, 320, 1, A, A, A), zq.ZQ_ERR_UNSUPPORTED),  # rotation: d % 128 == 0 or d == 192
     ((A + 4, 0, 4, 128, 0, A, A, A), zq.ZQ_ERR_ALIGN),
     ((A, 0, 4, 128, 0, A + 1, A, A), zq.ZQ_ERR_ALIGN),
     ((A, 0, 4, 128, 0, A, A, A + 8), zq.ZQ_ERR_ALIGN),

@@ -43,6 +43,18 @@ def test_quantize_bitwise_other_widths(n_vec, d):
     assert gds == rds and np.array_equal(g, r)
 
 
+@pytest.mark.parametrize("src", ["f32", "bf16"])
+@pytest.mark.parametrize("n_vec", [1, 333, 20000])
+def test_quantize_d192_rotation_bitwise(n_vec, src):
+    # MLA queries/keys: H128 on channels 0..127, sqrt2 * H64 on 128..191;
+    # one warp per vector, more vectors than the grid covers at 20000
+    x = torch.randn((n_vec, 192), generator=torch.Generator().manual_seed(n_vec)) * 2.0
+    x[0, 150] = 40.0  # an outlier in the 64-channel slice
+    g, gds, r, rds = _run(x, src, True)
+    assert gds == rds
+    assert np.array_equal(g, r), "%d of %d codes differ" % (int((g != r).sum()), g.size)
+
+
 def test_quantize_empty_and_zero():
     import bf16_causal_prefill_02_b200 as zq
 

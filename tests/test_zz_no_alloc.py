@@ -64,7 +64,7 @@ def test_noalloc_rejects_bad_arguments_like_the_regular_entry():
     out = torch.empty((4, 128), dtype=torch.uint8, device="cuda")
     s = torch.cuda.current_stream().cuda_stream
     assert zq.zq_quantize_fp8_noalloc(x.data_ptr(), 0, 4, 128, 0, out.data_ptr(), None, s) == zq.ZQ_ERR_NULL
-    assert zq.zq_quantize_fp8_noalloc(x.data_ptr(), 0, 4, 192, 1, out.data_ptr(), ds.data_ptr(), s) == zq.ZQ_ERR_UNSUPPORTED
+    assert zq.zq_quantize_fp8_noalloc(x.data_ptr(), 0, 4, 320, 1, out.data_ptr(), ds.data_ptr(), s) == zq.ZQ_ERR_UNSUPPORTED
     assert zq.zq_quantize_fp8_noalloc(x.data_ptr() + 4, 0, 4, 128, 0, out.data_ptr(), ds.data_ptr(), s) == zq.ZQ_ERR_ALIGN
     # empty input: only the descale (0) is written
     assert zq.zq_quantize_fp8_noalloc(None, 0, 0, 128, 0, None, ds.data_ptr(), s) == zq.ZQ_OK
