@@ -44,16 +44,17 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
 }
 
 // One bounded poll: the thread may sleep inside try_wait until the phase
-// completes or about `kSuspendNs` pass, so polling costs few issue slots.
-constexpr uint32_t kSuspendNs = 20000;
+// completes or a hardware-chosen time limit passes.  No suspend-time hint is
+// given: an explicit 20 us hint woke waiters late enough to cost the BF16
+// kernel about 5% at S = 16K, and 2 us was no better than none.
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar_addr), "r"(parity), "n"(kSuspendNs)
+      : "r"(bar_addr), "r"(parity)
       : "memory");
   return ok != 0;
 }
