@@ -17,6 +17,9 @@ Functions (all fp64 unless stated):
   attn_fp8_emul     R2  FP8 P path: per-(row, 64-key block) power-of-2 scale,
                         exact-exp2 or Lean P rounding, rounded-row-sum division
   quantize_fp8      R3  per-tensor amax quantiser, optional 128-point FWHT
+  quantize_fp8_grouped  R3 applied per (batch, group of heads): one scale
+                        per (batch, kv head), the flash_attn_func FP8 layout
+  dequant_grouped       codes times the per-(batch, head group) descale
   e4m3_decode/encode    OCP e4m3fn codec
   brute_attn            dense numpy softmax for tiny inputs (a cross-check)
 
@@ -154,6 +157,47 @@ def quantize_fp8(x: np.ndarray, hadamard: bool = False):
     if rc != 0:
         raise ValueError("zo_quantize_fp8 rejected the arguments")
     return out, np.float32(ds[0])
+
+
+def quantize_fp8_grouped(x: np.ndarray, heads_per_scale: int = 1, hadamard: bool = False):
+    """R3 with one scale per (batch, group of heads).
+
+    x: (B, S, H, d) float32, or uint16 holding bf16 bits.  The heads
+    [gi*heads_per_scale, (gi+1)*heads_per_scale) of batch b form slot
+    (b, gi); each slot, x[b, :, heads of gi, :], is quantised on its own
+    exactly as quantize_fp8 quantises a whole tensor (own amax, own descale).
+    With heads_per_scale = Hq / Hkv for queries and 1 for keys and values
+    this gives the (batch, kv head) descales of flash_attn_func's FP8
+    interface, which the pages name as the interface the kernel replaces
+    ([P2] "Che cosa ha annunciato Zyphra").
+
+    Returns (codes uint8 (B, S, H, d), descale float32 (B, H/heads_per_scale))."""
+    x = np.ascontiguousarray(x)
+    if x.ndim != 4:
+        raise ValueError("quantize_fp8_grouped takes x of shape (B, S, H, d)")
+    B, S, H, d = x.shape
+    g = int(heads_per_scale)
+    if g <= 0 or H % g != 0:
+        raise ValueError("heads_per_scale must divide H")
+    codes = np.zeros(x.shape, dtype=np.uint8)
+    ds = np.zeros((B, H // g), dtype=np.float32)
+    for b in range(B):
+        for gi in range(H // g):
+            sl = np.ascontiguousarray(x[b, :, gi * g:(gi + 1) * g, :])
+            c, dsc = quantize_fp8(sl, hadamard=hadamard)
+            codes[b, :, gi * g:(gi + 1) * g, :] = c
+            ds[b, gi] = dsc
+    return codes, ds
+
+
+def dequant_grouped(codes: np.ndarray, descale: np.ndarray) -> np.ndarray:
+    """codes (B, S, H, d) times descale (B, G) of head group h // (H / G),
+    exactly, in fp64."""
+    B, S, H, d = codes.shape
+    G = descale.shape[1]
+    val = e4m3_decode(codes)
+    per_head = np.repeat(np.asarray(descale, dtype=np.float64), H // G, axis=1)  # (B, H)
+    return val * per_head[:, None, :, None]
 
 
 # ------------------------------------------------------------- attention

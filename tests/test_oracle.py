@@ -349,3 +349,71 @@ def test_fp8_emulation_meets_tolerance_on_tiny(mode, tol):
     oe, _ = oracle.attn_fp8_emul(qd, kd, vd, mode=mode)
     err = oracle.rel_rmse(oe, o)
     assert err <= tol, err
+
+
+# --------------------------------------------- per-(batch, head group) scales
+def _grouped_input(B=2, S=40, H=6, d=128, seed=31):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((B, S, H, d)).astype(np.float32)
+    # heads far apart in magnitude, as separate kv heads can be
+    x *= np.float32(2.0) ** rng.integers(-6, 7, size=(B, 1, H, 1)).astype(np.float32)
+    return x
+
+
+@pytest.mark.parametrize("g", [1, 2, 3, 6])
+@pytest.mark.parametrize("hadamard", [False, True])
+def test_grouped_quantiser_slot_by_slot(g, hadamard):
+    x = _grouped_input()
+    codes, ds = oracle.quantize_fp8_grouped(x, heads_per_scale=g, hadamard=hadamard)
+    assert ds.shape == (2, 6 // g)
+    rot = oracle.fwht128(x) if hadamard else x
+    for b in range(2):
+        for gi in range(6 // g):
+            hs = slice(gi * g, (gi + 1) * g)
+            xs = rot[b, :, hs, :]
+            # the slot's own amax lands on +-448 and sets its descale
+            amax = np.float32(np.abs(xs).max())
+            assert (codes[b, :, hs, :] & 0x7F).max() == 0x7E
+            exp_ds = np.float32(amax / np.float32(448.0))
+            if hadamard:
+                exp_ds = np.float32(exp_ds * np.float32(2.0 ** -3.5))
+            assert ds[b, gi] == exp_ds
+            # codes are the torch e4m3 cast of the slot scaled by fl32(448/amax)
+            inv = np.float32(np.float32(448.0) / amax)
+            assert np.array_equal(codes[b, :, hs, :], _t2e4m3_codes((xs * inv).astype(np.float32)))
+
+
+def test_grouped_quantiser_power_of_two_touches_one_slot():
+    # scaling one slot's input by 2^5 multiplies its descale by 32 exactly
+    # and changes nothing else
+    x = _grouped_input()
+    c0, d0 = oracle.quantize_fp8_grouped(x, heads_per_scale=2)
+    y = x.copy()
+    y[1, :, 2:4, :] *= np.float32(32.0)
+    c1, d1 = oracle.quantize_fp8_grouped(y, heads_per_scale=2)
+    assert np.array_equal(c0, c1)
+    assert d1[1, 1] == np.float32(d0[1, 1] * np.float32(32.0))
+    mask = np.ones_like(d0, dtype=bool)
+    mask[1, 1] = False
+    assert np.array_equal(d0[mask], d1[mask])
+
+
+def test_grouped_quantiser_zero_slot_and_error_bound():
+    x = _grouped_input()
+    x[0, :, 0:3, :] = 0.0
+    codes, ds = oracle.quantize_fp8_grouped(x, heads_per_scale=3)
+    assert ds[0, 0] == 0.0 and not codes[0, :, 0:3, :].any()
+    deq = oracle.dequant_grouped(codes, ds)
+    # half an e4m3 step: relative 2^-4 for normals, 2^-10 descale below
+    # 2^-6 of the slot's range (subnormal spacing 2^-9)
+    per_head = np.repeat(ds.astype(np.float64), 3, axis=1)[:, None, :, None]
+    bound = np.maximum(np.abs(x) / 16.0, per_head * 2.0 ** -10) * 1.0001 + 1e-30
+    assert np.all(np.abs(deq - x) <= bound)
+
+
+def test_grouped_quantiser_one_slot_is_per_tensor():
+    # B = 1 with every head in one group is the per-tensor quantiser
+    x = _grouped_input(B=1, H=4)
+    c, d = oracle.quantize_fp8_grouped(x, heads_per_scale=4)
+    c1, d1 = oracle.quantize_fp8(x)
+    assert np.array_equal(c, c1) and d[0, 0] == d1
