@@ -25,6 +25,7 @@ HEADER_PATH = os.path.join(os.path.dirname(HERE), "include", "zattn.h")
 ZQ_DTYPE_BF16, ZQ_DTYPE_FP8_E4M3 = 0, 1
 ZQ_X_F32, ZQ_X_BF16 = 0, 1
 ZQ_SOFTMAX_EXACT, ZQ_SOFTMAX_LEANP = 0, 1
+ZQ_DESCALE_PER_TENSOR, ZQ_DESCALE_PER_KV_HEAD = 0, 1
 ZQ_OK, ZQ_ERR_NULL, ZQ_ERR_SHAPE, ZQ_ERR_UNSUPPORTED = 0, -1, -2, -3
 ZQ_ERR_ALIGN, ZQ_ERR_ARCH, ZQ_ERR_CUDA, ZQ_ERR_TIMEOUT = -4, -5, -6, -7
 
@@ -44,7 +45,7 @@ class zq_attn_args(ctypes.Structure):
         ("softmax_scale", ctypes.c_float), ("causal", ctypes.c_int), ("dtype", ctypes.c_int),
         ("q_descale", ctypes.c_void_p), ("k_descale", ctypes.c_void_p), ("v_descale", ctypes.c_void_p),
         ("softmax_mode", ctypes.c_int), ("block_scale", ctypes.c_int), ("headroom_T", ctypes.c_int),
-        ("status", ctypes.c_void_p),
+        ("status", ctypes.c_void_p), ("descale_layout", ctypes.c_int),
     ]
 
 
@@ -67,6 +68,10 @@ def _load():
     lib.zq_quantize_fp8.restype = i32
     lib.zq_quantize_fp8_noalloc.argtypes = [P, i32, i64, i32, i32, P, P, P]
     lib.zq_quantize_fp8_noalloc.restype = i32
+    lib.zq_quantize_fp8_grouped.argtypes = [P, i32, i32, i64, i32, i32, i32, i32, P, P, P, P]
+    lib.zq_quantize_fp8_grouped.restype = i32
+    lib.zq_quantize_grouped_workspace_bytes.argtypes = [i32, i32, i32]
+    lib.zq_quantize_grouped_workspace_bytes.restype = ctypes.c_size_t
     lib.zq_quantize_noalloc_scratch_bytes.argtypes = []
     lib.zq_quantize_noalloc_scratch_bytes.restype = ctypes.c_size_t
     lib.zq_debug_exp2.argtypes = [P, P, i64, i32, P]
@@ -119,6 +124,16 @@ def zq_quantize_fp8_noalloc(x, x_dtype, n_vec, d, hadamard, x_fp8, descale, stre
     fixed scratch array inside the library; calls that overlap on the GPU
     race.  The first call on a device sets up the array's address."""
     return _lib.zq_quantize_fp8_noalloc(x, x_dtype, n_vec, d, hadamard, x_fp8, descale, stream)
+
+
+def zq_quantize_fp8_grouped(x, x_dtype, B, S, H, d, heads_per_scale, hadamard, x_fp8, descale,
+                            workspace, stream) -> int:
+    return _lib.zq_quantize_fp8_grouped(x, x_dtype, B, S, H, d, heads_per_scale, hadamard, x_fp8,
+                                        descale, workspace, stream)
+
+
+def zq_quantize_grouped_workspace_bytes(B, H, heads_per_scale) -> int:
+    return int(_lib.zq_quantize_grouped_workspace_bytes(B, H, heads_per_scale))
 
 
 def zq_quantize_noalloc_scratch_bytes() -> int:
@@ -194,6 +209,51 @@ def quantize_fp8(x, hadamard: bool = False, out=None, descale=None, workspace=No
     return out, descale
 
 
+def quantize_fp8_grouped(x, heads_per_scale=1, hadamard: bool = False, out=None, descale=None,
+                         workspace=None, stream=None):
+    """e4m3 quantisation of a (B, S, H, d) CUDA tensor with one scale per
+    (batch, group of heads_per_scale heads).
+
+    Queries take heads_per_scale = Hq / Hkv, keys and values 1: the result
+    feeds attn_fwd with per-(batch, kv head) descales.  Returns (codes as
+    torch.float8_e4m3fn, descale fp32 tensor of shape (B, H / heads_per_scale))."""
+    torch = _torch()
+    if not x.is_cuda or not x.is_contiguous() or x.dim() != 4:
+        raise ValueError("x must be a contiguous (B, S, H, d) CUDA tensor")
+    if x.dtype == torch.float32:
+        xd = ZQ_X_F32
+    elif x.dtype == torch.bfloat16:
+        xd = ZQ_X_BF16
+    else:
+        raise TypeError("quantize_fp8_grouped takes float32 or bfloat16")
+    B, S, H, d = x.shape
+    g = int(heads_per_scale)
+    if g <= 0 or H % g != 0:
+        raise ValueError("heads_per_scale must divide the head count")
+    if out is None:
+        out = torch.empty(x.shape, dtype=torch.float8_e4m3fn, device=x.device)
+    if descale is None:
+        descale = torch.empty((B, H // g), dtype=torch.float32, device=x.device)
+    if workspace is None:
+        nbytes = zq_quantize_grouped_workspace_bytes(B, H, g)
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=x.device)
+    _check(zq_quantize_fp8_grouped(x.data_ptr(), xd, B, S, H, d, g, int(bool(hadamard)), out.data_ptr(),
+                                   descale.data_ptr(), workspace.data_ptr(), _stream(stream)),
+           "zq_quantize_fp8_grouped")
+    return out, descale
+
+
+def _descale_layout(B, Hkv, *descales) -> int:
+    """Per-tensor when every given descale holds one value, per-(batch, kv
+    head) when they hold B * Hkv values."""
+    sizes = {t.numel() for t in descales if t is not None}
+    if not sizes or sizes == {1}:
+        return ZQ_DESCALE_PER_TENSOR
+    if sizes == {B * Hkv}:
+        return ZQ_DESCALE_PER_KV_HEAD
+    raise ValueError("descales must all hold 1 or all hold B * Hkv values, got %s" % sorted(sizes))
+
+
 def attn_fwd(q, k, v, out=None, lse=None, softmax_scale=None, causal=True, q_descale=None,
              k_descale=None, v_descale=None, softmax_mode=ZQ_SOFTMAX_LEANP, block_scale=True,
              headroom_T=8, status=None, return_lse=True, stream=None, debug=None, debug_at=(0, 0),
@@ -201,7 +261,9 @@ def attn_fwd(q, k, v, out=None, lse=None, softmax_scale=None, causal=True, q_des
     """Causal prefill attention on CUDA tensors.
 
     q (B,Sq,Hq,d_qk), k (B,Sk,Hkv,d_qk), v (B,Sk,Hkv,d_v): bfloat16, or FP8
-    e4m3 (float8_e4m3fn / uint8) with per-tensor fp32 descale tensors.
+    e4m3 (float8_e4m3fn / uint8) with fp32 descale tensors: one value each
+    (per tensor) or B * Hkv values each (per batch and kv head, as
+    quantize_fp8_grouped returns them).
     Returns (out bf16 (B,Sq,Hq,d_v), lse fp32 (B,Hq,Sq) or None)."""
     torch = _torch()
     for t in (q, k, v):
@@ -230,6 +292,7 @@ def attn_fwd(q, k, v, out=None, lse=None, softmax_scale=None, causal=True, q_des
     a.block_scale = int(bool(block_scale))
     a.headroom_T = int(headroom_T)
     a.status = _ptr(status)
+    a.descale_layout = _descale_layout(B, Hkv, q_descale, k_descale, v_descale) if dtype == ZQ_DTYPE_FP8_E4M3 else 0
     if debug is not None:
         _check(zq_attn_fwd_debug(a, debug.data_ptr(), int(debug_at[0]), int(debug_at[1]), int(debug_flags),
                                  _stream(stream)), "zq_attn_fwd_debug")

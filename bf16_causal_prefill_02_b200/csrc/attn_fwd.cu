@@ -580,13 +580,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t col_h = (uint32_t)half * 64;
     const uint32_t lane_off = (uint32_t)(qd * 32 + sub * 16) << 16;  // 16-lane group
     constexpr unsigned kFull = 0xffffffffu;
-    float c = p.softmax_scale * 1.4426950408889634f;  // log2(e)
+    float c = p.softmax_scale * 1.4426950408889634f;  // log2(e); FP8: set per unit
     float vscale = 1.0f;
     if (DT == 1) {
-      const float qds = p.q_descale ? *p.q_descale : 1.0f;
-      const float kds = p.k_descale ? *p.k_descale : 1.0f;
-      vscale = p.v_descale ? *p.v_descale : 1.0f;
-      c = ((p.softmax_scale * qds) * kds) * 1.4426950408889634f;
       if (sub == 0) {
         // SFB (scales of V and of the ones matrix): all 2^0 = 0x7F; warp q
         // writes all 32 lanes of its quarter
@@ -644,6 +640,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     yref = -INFINITY;
     eref = kInvalidExp;
     l = 0.0f;
+    if (DT == 1) {
+      // dequantisation scales of this unit's (batch, kv head), or the
+      // per-tensor ones; the score scale folds q and k descales and log2(e)
+      const int di = p.descale_per_kv ? b * p.Hkv + wu.g : 0;
+      const float qds = p.q_descale ? p.q_descale[di] : 1.0f;
+      const float kds = p.k_descale ? p.k_descale[di] : 1.0f;
+      vscale = p.v_descale ? p.v_descale[di] : 1.0f;
+      c = ((p.softmax_scale * qds) * kds) * 1.4426950408889634f;
+    }
     for (int j = 0; ok && j < n_kv; ++j) {
       const int jg = jt + j;
       const int buf = jg & 1;

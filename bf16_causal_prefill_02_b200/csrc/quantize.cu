@@ -202,6 +202,191 @@ __global__ void __launch_bounds__(256) quant192_write_kernel(const void* __restr
   }
 }
 
+// ---------------------------------------------------------------------------
+// One scale per (batch, group of heads): x is (B, S, H, d) and the heads
+// [gi*g, gi*g + g) of batch b share slot b*(H/g) + gi, i.e. the per-(batch,
+// kv head) descales of flash_attn_func's FP8 interface.  The grid is
+// (chunks, slots): a CTA works inside one slot, so its maximum goes out in
+// a single atomicMax on the slot's word.  Each of a slot's S rows holds g*d
+// contiguous elements at ((b*S + s)*H + gi*g)*d.
+//   HM 0/1  items of 4 elements per thread (row length g*d, a multiple of
+//           8).  With the rotation (HM 1, d % 128 == 0) a row is a whole
+//           number of 128-slices and a warp's 32 consecutive items are one
+//           aligned slice, so fwht128_warp applies unchanged.
+//   HM 2    d = 192 with the rotation: one warp per 192-vector (g per row).
+// Items are visited by a grid-stride walk within the slot; the (row, item
+// in row) position advances by a fixed step without a division per item.
+struct ItemWalk {
+  int64_t row;
+  int col;
+  int64_t drow;
+  int dcol, ipr;
+  __device__ ItemWalk(int64_t k0, int64_t step, int ipr_) : ipr(ipr_) {
+    row = k0 / ipr_;
+    col = (int)(k0 % ipr_);
+    drow = step / ipr_;
+    dcol = (int)(step % ipr_);
+  }
+  __device__ __forceinline__ void next() {
+    row += drow;
+    col += dcol;
+    if (col >= ipr) {
+      col -= ipr;
+      ++row;
+    }
+  }
+};
+
+struct GroupGeo {
+  int64_t S;  // rows per slot
+  int H, d, g, gpb;  // heads, channels, heads per slot, slots per batch
+};
+
+__device__ __forceinline__ int64_t slot_base(const GroupGeo& G, int slot) {
+  const int b = slot / G.gpb, gi = slot % G.gpb;
+  return ((int64_t)b * G.S * G.H + (int64_t)gi * G.g) * G.d;
+}
+
+__device__ __forceinline__ float block_max_256(float m) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  __shared__ float red[8];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  float r = red[0];
+  for (int w = 1; w < (int)(blockDim.x >> 5); ++w) r = fmaxf(r, red[w]);
+  return r;
+}
+
+template <bool BF16IN, int HM>
+__global__ void __launch_bounds__(256) quantg_amax_kernel(const void* __restrict__ x, GroupGeo G,
+                                                          unsigned* __restrict__ amax_bits) {
+  const int lane = threadIdx.x & 31;
+  const int slot = blockIdx.y;
+  const int64_t base = slot_base(G, slot);
+  const int64_t rstride = (int64_t)G.H * G.d;
+  float m = 0.0f;
+  if constexpr (HM == 2) {
+    const int nw = blockDim.x >> 5;
+    ItemWalk w((int64_t)blockIdx.x * nw + (threadIdx.x >> 5), (int64_t)gridDim.x * nw, G.g);
+    for (; w.row < G.S; w.next()) {
+      const int64_t v0 = base + w.row * rstride + (int64_t)w.col * 192;
+      float a[4], c[2];
+      load4<BF16IN>(x, v0 + 4 * lane, a);
+      load2<BF16IN>(x, v0 + 128 + 2 * lane, c);
+      fwht128_warp(a, lane);
+      fwht64x2_warp_scaled(c, lane);
+      m = fmaxf(m, fmaxf(fmaxf(fabsf(a[0]), fabsf(a[1])), fmaxf(fabsf(a[2]), fabsf(a[3]))));
+      m = fmaxf(m, fmaxf(fabsf(c[0]), fabsf(c[1])));
+    }
+  } else {
+    ItemWalk w((int64_t)blockIdx.x * blockDim.x + threadIdx.x, (int64_t)gridDim.x * blockDim.x,
+               G.g * G.d / 4);
+    for (; w.row < G.S; w.next()) {
+      float v[4];
+      load4<BF16IN>(x, base + w.row * rstride + 4 * (int64_t)w.col, v);
+      if constexpr (HM == 1) fwht128_warp(v, lane);
+      m = fmaxf(m, fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3]))));
+    }
+  }
+  const float r = block_max_256(m);
+  if (threadIdx.x == 0) atomicMax(amax_bits + slot, __float_as_uint(r));
+}
+
+__device__ __forceinline__ uint32_t e4m3x4(const float (&v)[4], float inv) {
+  const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(
+      make_float2(__fmul_rn(v[0], inv), __fmul_rn(v[1], inv)), __NV_SATFINITE, __NV_E4M3);
+  const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(
+      make_float2(__fmul_rn(v[2], inv), __fmul_rn(v[3], inv)), __NV_SATFINITE, __NV_E4M3);
+  return (uint32_t)lo | ((uint32_t)hi << 16);
+}
+
+template <bool BF16IN, int HM>
+__global__ void __launch_bounds__(256) quantg_write_kernel(const void* __restrict__ x, GroupGeo G,
+                                                           const unsigned* __restrict__ amax_bits,
+                                                           uint8_t* __restrict__ out,
+                                                           float* __restrict__ descale) {
+  const int lane = threadIdx.x & 31;
+  const int slot = blockIdx.y;
+  const float amax = __uint_as_float(amax_bits[slot]);
+  const float inv = amax > 0.0f ? __fdiv_rn(448.0f, amax) : 1.0f;
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    float ds = __fdiv_rn(amax, 448.0f);
+    if (HM != 0) ds = __fmul_rn(ds, 0.08838834764831845f);  // fl32(2^-3.5)
+    descale[slot] = ds;
+  }
+  const int64_t base = slot_base(G, slot);
+  const int64_t rstride = (int64_t)G.H * G.d;
+  if constexpr (HM == 2) {
+    const int nw = blockDim.x >> 5;
+    ItemWalk w((int64_t)blockIdx.x * nw + (threadIdx.x >> 5), (int64_t)gridDim.x * nw, G.g);
+    for (; w.row < G.S; w.next()) {
+      const int64_t v0 = base + w.row * rstride + (int64_t)w.col * 192;
+      float a[4], c[2];
+      load4<BF16IN>(x, v0 + 4 * lane, a);
+      load2<BF16IN>(x, v0 + 128 + 2 * lane, c);
+      fwht128_warp(a, lane);
+      fwht64x2_warp_scaled(c, lane);
+      *reinterpret_cast<uint32_t*>(out + v0 + 4 * lane) = e4m3x4(a, inv);
+      const __nv_fp8x2_storage_t t = __nv_cvt_float2_to_fp8x2(
+          make_float2(__fmul_rn(c[0], inv), __fmul_rn(c[1], inv)), __NV_SATFINITE, __NV_E4M3);
+      *reinterpret_cast<uint16_t*>(out + v0 + 128 + 2 * lane) = (uint16_t)t;
+    }
+  } else {
+    ItemWalk w((int64_t)blockIdx.x * blockDim.x + threadIdx.x, (int64_t)gridDim.x * blockDim.x,
+               G.g * G.d / 4);
+    for (; w.row < G.S; w.next()) {
+      const int64_t i = base + w.row * rstride + 4 * (int64_t)w.col;
+      float v[4];
+      load4<BF16IN>(x, i, v);
+      if constexpr (HM == 1) fwht128_warp(v, lane);
+      *reinterpret_cast<uint32_t*>(out + i) = e4m3x4(v, inv);
+    }
+  }
+}
+
+// Host-side launcher of the grouped quantiser; arguments were validated by
+// the caller (B, H >= 1, S >= 0, H % g == 0, B*H/g <= 65535).
+cudaError_t launch_quantize_grouped(const void* x, int x_bf16, int B, int64_t S, int H, int d, int g,
+                                    int hadamard, void* out, float* descale, void* workspace,
+                                    cudaStream_t st, int num_sms) {
+  unsigned* amax = static_cast<unsigned*>(workspace);
+  GroupGeo G;
+  G.S = S;
+  G.H = H;
+  G.d = d;
+  G.g = g;
+  G.gpb = H / g;
+  const int n_slots = B * G.gpb;
+  cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(unsigned) * (size_t)n_slots, st);
+  if (e != cudaSuccess) return e;
+  const int threads = 256;
+  // items per slot, in the unit one thread (HM 0/1) or one warp (HM 2) takes
+  const int64_t items = hadamard == 2 ? S * g : S * (int64_t)(g * d / 4);
+  const int64_t per_cta = hadamard == 2 ? threads / 32 : threads;
+  const int64_t useful = (items + per_cta - 1) / per_cta;
+  const int64_t want = ((int64_t)num_sms * 8 + n_slots - 1) / n_slots;
+  int cps = (int)(want < useful ? want : useful);
+  if (cps < 1) cps = 1;
+  const dim3 grid(cps, n_slots);
+#define ZQ_QUANTG_LAUNCH(BF, HM_)                                                                 \
+  do {                                                                                            \
+    quantg_amax_kernel<BF, HM_><<<grid, threads, 0, st>>>(x, G, amax);                            \
+    quantg_write_kernel<BF, HM_><<<grid, threads, 0, st>>>(x, G, amax, (uint8_t*)out, descale);   \
+  } while (0)
+  if (x_bf16) {
+    if (hadamard == 2) ZQ_QUANTG_LAUNCH(true, 2);
+    else if (hadamard) ZQ_QUANTG_LAUNCH(true, 1);
+    else ZQ_QUANTG_LAUNCH(true, 0);
+  } else {
+    if (hadamard == 2) ZQ_QUANTG_LAUNCH(false, 2);
+    else if (hadamard) ZQ_QUANTG_LAUNCH(false, 1);
+    else ZQ_QUANTG_LAUNCH(false, 0);
+  }
+#undef ZQ_QUANTG_LAUNCH
+  return cudaGetLastError();
+}
+
 // Host-side launcher; arguments were validated by the caller.
 cudaError_t launch_quantize(const void* x, int x_bf16, int64_t n, int hadamard, void* out,
                             float* descale, void* workspace, cudaStream_t st, int num_sms) {

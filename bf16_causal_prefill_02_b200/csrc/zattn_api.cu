@@ -15,6 +15,7 @@ namespace {
 
 constexpr int kVersion = 100;  // 0.1.0
 constexpr uint64_t kTimeoutNs = 2000000000ull;  // bound on any single device-side wait
+constexpr int64_t kMaxGroupedSlots = 65535;      // grouped quantiser: slots are grid.y
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -47,6 +48,8 @@ int validate_attn(const zq_attn_args* a) {
       return ZQ_ERR_UNSUPPORTED;
     if (a->block_scale != 0 && a->block_scale != 1) return ZQ_ERR_UNSUPPORTED;
     if (a->headroom_T < 0 || a->headroom_T > 8) return ZQ_ERR_UNSUPPORTED;
+    if (a->descale_layout != ZQ_DESCALE_PER_TENSOR && a->descale_layout != ZQ_DESCALE_PER_KV_HEAD)
+      return ZQ_ERR_UNSUPPORTED;
   }
   if (!(std::isfinite(a->softmax_scale))) return ZQ_ERR_SHAPE;
   // grid = n_qtiles * B * Hq blocks; TMA element counts and strides
@@ -102,6 +105,8 @@ static int attn_impl(const zq_attn_args* a, void* dbg, int dbg_bh, int dbg_t, in
   L.p.q_descale = a->q_descale;
   L.p.k_descale = a->k_descale;
   L.p.v_descale = a->v_descale;
+  L.p.descale_per_kv =
+      a->dtype == ZQ_DTYPE_FP8_E4M3 && a->descale_layout == ZQ_DESCALE_PER_KV_HEAD ? 1 : 0;
   L.p.status = a->status;
   L.p.B = a->B;
   L.p.Sq = a->Sq;
@@ -173,6 +178,7 @@ int zq_attn_fwd(const void* q, const void* k, const void* v, void* out, float* l
   a.block_scale = 1;
   a.headroom_T = 8;
   a.status = nullptr;
+  a.descale_layout = ZQ_DESCALE_PER_TENSOR;
   return zq_attn_fwd_ex(&a, stream);
 }
 
@@ -221,6 +227,37 @@ int zq_quantize_fp8_noalloc(const void* x, int x_dtype, int64_t n_vec, int d, in
 }
 
 size_t zq_quantize_noalloc_scratch_bytes(void) { return zq::noalloc_scratch_capacity(); }
+
+size_t zq_quantize_grouped_workspace_bytes(int B, int H, int heads_per_scale) {
+  if (B <= 0 || H <= 0 || heads_per_scale <= 0 || H % heads_per_scale != 0) return 0;
+  const int64_t slots = (int64_t)B * (H / heads_per_scale);
+  if (slots > kMaxGroupedSlots) return 0;
+  return (size_t)((slots * 4 + 15) / 16 * 16);
+}
+
+int zq_quantize_fp8_grouped(const void* x, int x_dtype, int B, int64_t S, int H, int d,
+                            int heads_per_scale, int hadamard, void* x_fp8, float* descale,
+                            void* workspace, void* stream) {
+  if (!descale || !workspace) return ZQ_ERR_NULL;
+  if (B <= 0 || H <= 0 || S < 0 || d <= 0 || heads_per_scale <= 0) return ZQ_ERR_SHAPE;
+  if (H % heads_per_scale != 0) return ZQ_ERR_SHAPE;
+  if ((int64_t)B * (H / heads_per_scale) > kMaxGroupedSlots) return ZQ_ERR_SHAPE;
+  if (S > 0 && (!x || !x_fp8)) return ZQ_ERR_NULL;
+  if (x_dtype != ZQ_X_F32 && x_dtype != ZQ_X_BF16) return ZQ_ERR_UNSUPPORTED;
+  if (d % 8 != 0 || (hadamard && d % 128 != 0 && d != 192)) return ZQ_ERR_UNSUPPORTED;
+  if (S > ((int64_t)1 << 40) || (int64_t)H * d > ((int64_t)1 << 24) ||
+      (int64_t)B * S > ((int64_t)1 << 40) / ((int64_t)H * d))
+    return ZQ_ERR_SHAPE;
+  if (!aligned16(x) || !aligned16(x_fp8) || !aligned16(workspace)) return ZQ_ERR_ALIGN;
+  int sms = 0;
+  int rc = check_device(&sms);
+  if (rc != ZQ_OK) return rc;
+  cudaError_t e = zq::launch_quantize_grouped(
+      x, x_dtype == ZQ_X_BF16, B, S, H, d, heads_per_scale,
+      hadamard ? (d % 128 == 0 ? 1 : 2) : 0, x_fp8, descale, workspace,
+      static_cast<cudaStream_t>(stream), sms);
+  return e == cudaSuccess ? ZQ_OK : ZQ_ERR_CUDA;
+}
 
 int zq_debug_exp2(const float* x, float* y, int64_t n, int degree, void* stream) {
   if (n < 0) return ZQ_ERR_SHAPE;

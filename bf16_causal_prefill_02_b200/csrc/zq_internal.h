@@ -13,6 +13,9 @@ struct AttnParams {
   const float* q_descale;
   const float* k_descale;
   const float* v_descale;
+  // 0: each descale pointer holds one fp32; 1: each holds B * Hkv fp32,
+  // entry b * Hkv + kv_head (query head h uses kv head h / (Hq / Hkv))
+  int descale_per_kv;
   int* status;
   int B, Sq, Sk, Hq, Hkv;
   int n_qtiles;
@@ -52,6 +55,11 @@ cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t st);
 // rotation (H128 on channels 0..127, sqrt2 * H64 on 128..191)
 cudaError_t launch_quantize(const void* x, int x_bf16, int64_t n, int hadamard, void* out,
                             float* descale, void* workspace, cudaStream_t st, int num_sms);
+// x (B, S, H, d); heads [gi*g, gi*g + g) of batch b share one scale, slot
+// b*(H/g) + gi; hadamard as for launch_quantize.
+cudaError_t launch_quantize_grouped(const void* x, int x_bf16, int B, int64_t S, int H, int d, int g,
+                                    int hadamard, void* out, float* descale, void* workspace,
+                                    cudaStream_t st, int num_sms);
 void* noalloc_scratch_for_device(int dev);
 cudaError_t launch_exp2_check(const float* x, float* y, int64_t n, int degree, cudaStream_t st);
 size_t noalloc_scratch_capacity();

@@ -49,6 +49,10 @@ extern "C" {
 #define ZQ_SOFTMAX_EXACT 0 /* P~ = e4m3_rne(exp2(y - e))                   */
 #define ZQ_SOFTMAX_LEANP 1 /* P~ bits = clamp(rne(8 (y - e)) + 56, 0, 126) */
 
+/* ---- FP8 descale layouts (zq_attn_args.descale_layout) ---- */
+#define ZQ_DESCALE_PER_TENSOR 0  /* q/k/v_descale each point to one fp32        */
+#define ZQ_DESCALE_PER_KV_HEAD 1 /* each points to B * Hkv fp32, [b * Hkv + g] */
+
 /* ---- status codes ---- */
 #define ZQ_OK 0
 #define ZQ_ERR_NULL (-1)        /* a required pointer is NULL              */
@@ -78,7 +82,8 @@ extern "C" {
  *   (bottom-right alignment); a query row with no visible key gets out = 0,
  *   lse = -inf.
  *   q/k/v_descale: device pointers to one fp32 each (per-tensor dequant
- *   scale, FP8 only; NULL means 1.0); ignored for bf16.
+ *   scale, FP8 only; NULL means 1.0); ignored for bf16.  Per-(batch, kv
+ *   head) descales go through zq_attn_fwd_ex (descale_layout).
  *   FP8 uses Lean P with per-(row, 64-key block) power-of-2 scaling and
  *   headroom 8 (see zq_attn_fwd_ex for the other modes).
  * Errors: ZQ_ERR_NULL (q, k, v or out NULL), ZQ_ERR_SHAPE, ZQ_ERR_UNSUPPORTED,
@@ -121,6 +126,16 @@ typedef struct zq_attn_args {
    * that runs out writes ZQ_ERR_TIMEOUT there and the kernel returns early
    * (outputs are then undefined).  NULL: not reported. */
   int* status;
+  /* FP8 only.  ZQ_DESCALE_PER_TENSOR (0): q/k/v_descale each point to one
+   * fp32.  ZQ_DESCALE_PER_KV_HEAD (1): each points to B * Hkv fp32, row-major
+   * (batch, kv head); query head h of batch b is dequantised with
+   * q_descale[b * Hkv + h / (Hq / Hkv)], and its keys and values with the
+   * k_descale / v_descale entry of the same index.  This is the (batch,
+   * kv head) descale shape of flash_attn_func's FP8 interface, which the
+   * kernel is a drop-in for [P2 "Che cosa ha annunciato Zyphra"];
+   * zq_quantize_fp8_grouped produces such scales.  NULL pointers still
+   * mean 1.0. */
+  int descale_layout;
 } zq_attn_args;
 
 /* zq_attn_fwd_ex -- zq_attn_fwd with the options above.  Same errors, plus
@@ -205,6 +220,37 @@ ZQ_API int zq_quantize_fp8_noalloc(const void* x, int x_dtype, int64_t n_vec, in
 
 /* Capacity in bytes of the fixed scratch array of zq_quantize_fp8_noalloc. */
 ZQ_API size_t zq_quantize_noalloc_scratch_bytes(void);
+
+/*
+ * zq_quantize_fp8_grouped -- the quantiser of zq_quantize_fp8 with one scale
+ * per (batch, group of heads) instead of one per tensor.
+ *
+ *   x        (B, S, H, d) contiguous, fp32 or bf16 (x_dtype)
+ *   heads_per_scale  g: heads [gi*g, gi*g + g) of batch b form slot
+ *            b * (H / g) + gi.  Queries take g = Hq / Hkv and keys and
+ *            values g = 1, which gives the ZQ_DESCALE_PER_KV_HEAD layout of
+ *            zq_attn_args.
+ *   Each slot, x[b, :, heads of the slot, :], is quantised exactly as
+ *   zq_quantize_fp8 quantises a whole tensor (same rotation, same rounding,
+ *   its own amax): codes bit-identical to zq_quantize_fp8 run on that slot
+ *   alone.
+ *   x_fp8    (B, S, H, d) e4m3 bytes
+ *   descale  B * (H / g) fp32, row-major (batch, slot)
+ *   workspace  device scratch of zq_quantize_grouped_workspace_bytes(B, H, g)
+ *            bytes, 16-byte aligned, not shared with a concurrent call.
+ * S == 0 writes only the descales (0); x and x_fp8 may then be NULL.
+ * Errors: ZQ_ERR_NULL, ZQ_ERR_SHAPE (B, H, d, g <= 0, S < 0, H % g != 0,
+ *   more than 65535 slots, size overflow), ZQ_ERR_UNSUPPORTED (as for
+ *   zq_quantize_fp8), ZQ_ERR_ALIGN (x, x_fp8, workspace), ZQ_ERR_ARCH,
+ *   ZQ_ERR_CUDA.
+ */
+ZQ_API int zq_quantize_fp8_grouped(const void* x, int x_dtype, int B, int64_t S, int H, int d,
+                                   int heads_per_scale, int hadamard, void* x_fp8, float* descale,
+                                   void* workspace, void* stream);
+
+/* Bytes of device scratch zq_quantize_fp8_grouped needs for these sizes
+ * (4 per slot, rounded up to 16); 0 for arguments it would reject. */
+ZQ_API size_t zq_quantize_grouped_workspace_bytes(int B, int H, int heads_per_scale);
 
 /* zq_debug_exp2 -- y[i] = 2^x[i] by the kernels' software exp2 (degree 3 or
  * 4 minimax polynomial after range reduction), by CUDA's exp2f (degree 0) or

@@ -30,10 +30,11 @@ LSE_FLIP_FRAC = 5e-3
 
 class Case:
     def __init__(self, B, Sq, Sk, Hq, Hkv, dqk, dv, dtype="bf16", causal=True, block_scale=True,
-                 T=8, hadamard=False, seed=0, std=1.0, inputs=None):
+                 T=8, hadamard=False, seed=0, std=1.0, inputs=None, per_kv_descale=False):
         self.B, self.Sq, self.Sk, self.Hq, self.Hkv, self.dqk, self.dv = B, Sq, Sk, Hq, Hkv, dqk, dv
         self.dtype, self.causal, self.block_scale, self.T = dtype, causal, block_scale, T
         self.hadamard, self.seed, self.std = hadamard, seed, std
+        self.per_kv_descale = per_kv_descale
         if inputs is None:
             inputs = workloads.make_custom(B, Sq, Sk, Hq, Hkv, dqk, dv, seed=seed, std=std)
         self.q32, self.k32, self.v32 = (t.contiguous() for t in inputs)
@@ -48,6 +49,18 @@ class Case:
         if not self.fp8:
             self.qb, self.kb, self.vb = (t.to(torch.bfloat16) for t in (self.q32, self.k32, self.v32))
             self.qd, self.kd, self.vd = (t.to(torch.float64).numpy() for t in (self.qb, self.kb, self.vb))
+            return
+        if self.per_kv_descale:
+            # one scale per (batch, kv head): the query heads of a kv head
+            # share theirs
+            enc = []
+            for t, g, rot in ((self.q32, self.Hq // self.Hkv, self.hadamard), (self.k32, 1, self.hadamard),
+                              (self.v32, 1, False)):
+                enc.append(oracle.quantize_fp8_grouped(t.numpy(), heads_per_scale=g, hadamard=rot))
+            (self.cq, self.dsq), (self.ck, self.dsk), (self.cv, self.dsv) = enc
+            self.qd = oracle.dequant_grouped(self.cq, self.dsq)
+            self.kd = oracle.dequant_grouped(self.ck, self.dsk)
+            self.vd = oracle.dequant_grouped(self.cv, self.dsv)
             return
         enc = []
         for t, rot in ((self.q32, self.hadamard), (self.k32, self.hadamard), (self.v32, False)):
@@ -68,7 +81,8 @@ class Case:
             return zq.attn_fwd(q, k, v, causal=self.causal, debug=debug, debug_at=debug_at, status=status,
                                out=out, lse=lse, debug_flags=debug_flags)
         q, k, v = (torch.from_numpy(c).to(dev).view(torch.float8_e4m3fn) for c in (self.cq, self.ck, self.cv))
-        dq, dk, dv = (torch.tensor([float(d)], dtype=torch.float32, device=dev) for d in (self.dsq, self.dsk, self.dsv))
+        dq, dk, dv = (torch.tensor(np.asarray(d, dtype=np.float32).reshape(-1), device=dev)
+                      for d in (self.dsq, self.dsk, self.dsv))
         mode = zq.ZQ_SOFTMAX_EXACT if self.dtype == "exact" else zq.ZQ_SOFTMAX_LEANP
         return zq.attn_fwd(q, k, v, causal=self.causal, q_descale=dq, k_descale=dk, v_descale=dv,
                            softmax_mode=mode, block_scale=self.block_scale, headroom_T=self.T,

@@ -149,6 +149,34 @@ def test_fp8_hadamard_mla_192(dtype):
     check_against_oracle(Case(1, 400, 400, 2, 2, 192, 128, dtype=dtype, hadamard=True, inputs=(q, k, v)))
 
 
+@pytest.mark.parametrize("dtype", ["exact", "leanp"])
+@pytest.mark.parametrize("dqk,had", [(128, False), (128, True), (192, True)])
+def test_per_kv_head_descales(dtype, dqk, had):
+    # one descale per (batch, kv head) for q, k and v; heads whose inputs
+    # differ by powers of two up to 2^12 each get their own scale, and each
+    # CTA must pick the entry of its own unit (persistent CTAs cross batches
+    # and kv heads)
+    B, S, Hq, Hkv = 2, 450, 8, 2
+    q, k, v = workloads.make_custom(B, S, S, Hq, Hkv, dqk, 128, seed=40 + dqk)
+    q[0, :, 0:4] *= 64.0
+    k[1, :, 1] *= 1.0 / 64.0
+    v[0, :, 1] *= 0.01
+    v[1, :, 0] *= 50.0
+    c = Case(B, S, S, Hq, Hkv, dqk, 128, dtype=dtype, hadamard=had, inputs=(q, k, v), per_kv_descale=True)
+    assert c.dsq.shape == (B, Hkv) and len(set(c.dsv.ravel().tolist())) == B * Hkv
+    check_against_oracle(c)
+
+
+def test_per_kv_head_descales_many_units():
+    # short rows, 2 x 40 heads: persistent CTAs take units of many (batch,
+    # kv head) pairs in turn
+    q, k, v = workloads.make_custom(2, 300, 300, 40, 8, 128, 128, seed=44)
+    scale = torch.pow(2.0, torch.arange(-4, 4).float())[None, None, :, None]
+    c = Case(2, 300, 300, 40, 8, 128, 128, dtype="leanp", inputs=(q, k * scale, v / scale),
+             per_kv_descale=True)
+    check_against_oracle(c)
+
+
 @pytest.mark.parametrize("dtype", ["bf16", "leanp"])
 def test_large_logits_lazy_rescale(dtype):
     # scores growing along the sequence force the reference max / exponent

@@ -36,7 +36,8 @@ def _args(**kw):
     a = zq.zq_attn_args()
     d = dict(q=A, k=A, v=A, out=A, lse=None, B=1, Sq=128, Sk=128, Hq=2, Hkv=1, d_qk=128, d_v=128,
              softmax_scale=0.0, causal=1, dtype=zq.ZQ_DTYPE_BF16, q_descale=None, k_descale=None,
-             v_descale=None, softmax_mode=zq.ZQ_SOFTMAX_LEANP, block_scale=1, headroom_T=8, status=None)
+             v_descale=None, softmax_mode=zq.ZQ_SOFTMAX_LEANP, block_scale=1, headroom_T=8, status=None,
+             descale_layout=0)
     d.update(kw)
     for k, v in d.items():
         setattr(a, k, v)
@@ -61,6 +62,8 @@ def _args(**kw):
     (dict(dtype=1, block_scale=2), zq.ZQ_ERR_UNSUPPORTED),
     (dict(dtype=1, headroom_T=9), zq.ZQ_ERR_UNSUPPORTED),
     (dict(dtype=1, headroom_T=-1), zq.ZQ_ERR_UNSUPPORTED),
+    (dict(dtype=1, descale_layout=2), zq.ZQ_ERR_UNSUPPORTED),
+    (dict(dtype=1, descale_layout=-1), zq.ZQ_ERR_UNSUPPORTED),
     (dict(q=A + 8), zq.ZQ_ERR_ALIGN),
     (dict(out=A + 2), zq.ZQ_ERR_ALIGN),
     (dict(lse=A + 4), zq.ZQ_ERR_ALIGN),
@@ -96,6 +99,53 @@ def test_attn_plain_entry_validates_too():
 def test_quantize_argument_errors(args, code):
     x, xd, n, d, had, out, ds, ws = args
     assert zq.zq_quantize_fp8(x, xd, n, d, had, out, ds, ws, None) == code
+
+
+@pytest.mark.parametrize("args,code", [
+    # x, x_dtype, B, S, H, d, heads_per_scale, hadamard, x_fp8, descale, workspace
+    ((A, 0, 2, 10, 8, 128, 2, 0, A, None, A), zq.ZQ_ERR_NULL),
+    ((A, 0, 2, 10, 8, 128, 2, 0, A, A, None), zq.ZQ_ERR_NULL),
+    ((None, 0, 2, 10, 8, 128, 2, 0, A, A, A), zq.ZQ_ERR_NULL),
+    ((A, 0, 2, 10, 8, 128, 2, 0, None, A, A), zq.ZQ_ERR_NULL),
+    ((A, 0, 0, 10, 8, 128, 2, 0, A, A, A), zq.ZQ_ERR_SHAPE),
+    ((A, 0, 2, -1, 8, 128, 2, 0, A, A, A), zq.ZQ_ERR_SHAPE),
+    ((A, 0, 2, 10, 0, 128, 1, 0, A, A, A), zq.ZQ_ERR_SHAPE),
+    ((A, 0, 2, 10, 8, 0, 2, 0, A, A, A), zq.ZQ_ERR_SHAPE),
+    ((A, 0, 2, 10, 8, 128, 0, 0, A, A, A), zq.ZQ_ERR_SHAPE),
+    ((A, 0, 2, 10, 8, 128, 3, 0, A, A, A), zq.ZQ_ERR_SHAPE),      # H % g != 0
+    ((A, 0, 70000, 10, 1, 128, 1, 0, A, A, A), zq.ZQ_ERR_SHAPE),  # > 65535 slots
+    ((A, 2, 2, 10, 8, 128, 2, 0, A, A, A), zq.ZQ_ERR_UNSUPPORTED),
+    ((A, 0, 2, 10, 8, 12, 2, 0, A, A, A), zq.ZQ_ERR_UNSUPPORTED),
+    ((A, 0, 2, 10, 8, 320, 2, 1, A, A, A), zq.ZQ_ERR_UNSUPPORTED),
+    ((A + 4, 0, 2, 10, 8, 128, 2, 0, A, A, A), zq.ZQ_ERR_ALIGN),
+    ((A, 0, 2, 10, 8, 128, 2, 0, A + 1, A, A), zq.ZQ_ERR_ALIGN),
+    ((A, 0, 2, 10, 8, 128, 2, 0, A, A, A + 8), zq.ZQ_ERR_ALIGN),
+])
+def test_quantize_grouped_argument_errors(args, code):
+    assert zq.zq_quantize_fp8_grouped(*args, None) == code
+
+
+def test_quantize_grouped_workspace_bytes():
+    assert zq.zq_quantize_grouped_workspace_bytes(2, 8, 4) == 16     # 4 slots
+    assert zq.zq_quantize_grouped_workspace_bytes(3, 8, 1) == 96     # 24 slots
+    assert zq.zq_quantize_grouped_workspace_bytes(1, 5, 1) == 32     # 5 slots, rounded up
+    assert zq.zq_quantize_grouped_workspace_bytes(2, 8, 3) == 0      # g does not divide H
+    assert zq.zq_quantize_grouped_workspace_bytes(0, 8, 1) == 0
+    assert zq.zq_quantize_grouped_workspace_bytes(70000, 1, 1) == 0  # too many slots
+
+
+def test_descale_layout_from_tensor_sizes():
+    import torch
+
+    one, per = torch.ones(1), torch.ones(2 * 4)
+    assert zq._descale_layout(2, 4, None, None, None) == zq.ZQ_DESCALE_PER_TENSOR
+    assert zq._descale_layout(2, 4, one, one, None) == zq.ZQ_DESCALE_PER_TENSOR
+    assert zq._descale_layout(2, 4, per, per, per) == zq.ZQ_DESCALE_PER_KV_HEAD
+    assert zq._descale_layout(2, 4, per, None, per) == zq.ZQ_DESCALE_PER_KV_HEAD
+    with pytest.raises(ValueError):
+        zq._descale_layout(2, 4, one, per, per)
+    with pytest.raises(ValueError):
+        zq._descale_layout(2, 4, torch.ones(3), None, None)
 
 
 def test_no_cpu_fallback_without_library(tmp_path, monkeypatch):

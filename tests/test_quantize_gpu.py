@@ -95,3 +95,46 @@ def test_quantize_repeatable():
     c0 = outs[0][0].view(torch.uint8)
     for c, d in outs[1:]:
         assert torch.equal(c.view(torch.uint8), c0) and torch.equal(d, outs[0][1])
+
+
+@pytest.mark.parametrize("B,S,H,d,g,src,hadamard", [
+    (2, 300, 8, 128, 4, "f32", False),    # queries of 8:2 GQA
+    (2, 300, 8, 128, 1, "bf16", True),    # keys, rotated
+    (1, 257, 4, 192, 2, "f32", True),     # MLA width, d = 192 rotation
+    (2, 50, 16, 192, 4, "bf16", True),
+    (2, 100, 6, 192, 3, "bf16", False),   # rows not a whole number of 128-slices
+    (3, 1, 2, 64, 1, "f32", False),
+    (1, 1000, 32, 128, 8, "f32", True),   # more items than the grid covers
+    (4, 17, 3, 8, 3, "f32", False),
+])
+def test_quantize_grouped_bitwise(B, S, H, d, g, src, hadamard):
+    # one scale per (batch, group of g heads): codes and descales bit-identical
+    # to the oracle, which quantises each slot as a tensor of its own
+    import bf16_causal_prefill_02_b200 as zq
+
+    gen = torch.Generator().manual_seed(B * 1000 + S + H + d + g)
+    x = torch.randn((B, S, H, d), generator=gen)
+    # heads far apart in magnitude, so that every slot has its own scale
+    x *= torch.pow(2.0, torch.randint(-6, 7, (B, 1, H, 1), generator=gen).float())
+    if src == "bf16":
+        xb = x.to(torch.bfloat16)
+        ref_in = xb.view(torch.int16).numpy().view(np.uint16)
+        xg = xb.cuda()
+    else:
+        ref_in = x.numpy()
+        xg = x.cuda()
+    codes, ds = zq.quantize_fp8_grouped(xg, heads_per_scale=g, hadamard=hadamard)
+    torch.cuda.synchronize()
+    rc, rds = oracle.quantize_fp8_grouped(ref_in, heads_per_scale=g, hadamard=hadamard)
+    assert tuple(ds.shape) == (B, H // g)
+    assert np.array_equal(ds.cpu().numpy(), rds)
+    got = codes.view(torch.uint8).cpu().numpy()
+    assert np.array_equal(got, rc), "%d of %d codes differ" % (int((got != rc).sum()), rc.size)
+
+
+def test_quantize_grouped_empty_sequence():
+    import bf16_causal_prefill_02_b200 as zq
+
+    codes, ds = zq.quantize_fp8_grouped(torch.zeros((2, 0, 4, 128), device="cuda"), heads_per_scale=2)
+    torch.cuda.synchronize()
+    assert codes.numel() == 0 and ds.shape == (2, 2) and not ds.cpu().any()
