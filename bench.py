@@ -52,6 +52,8 @@ def parse():
     ap.add_argument("--S", type=int, default=None)
     ap.add_argument("--dtype", default="leanp", choices=["leanp", "exact", "bf16"])
     ap.add_argument("--hadamard", action="store_true")
+    ap.add_argument("--descale", default="tensor", choices=["tensor", "kv"],
+                    help="FP8 scales: one per tensor, or one per (batch, kv head)")
     ap.add_argument("--T", type=int, default=8, help="FP8 headroom T (block maximum lands in (2^(T-1), 2^T])")
     ap.add_argument("--no-energy", action="store_true", help="skip the attention-only power measurement")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -192,10 +194,12 @@ def load_traffic(key: str):
 class Step:
     """The hot path for one workload on one GPU; inputs resident in HBM."""
 
-    def __init__(self, w: workloads.Workload, dtype: str, hadamard: bool, seed_offset: int = 0, T: int = 8):
+    def __init__(self, w: workloads.Workload, dtype: str, hadamard: bool, seed_offset: int = 0, T: int = 8,
+                 per_kv: bool = False):
         import bf16_causal_prefill_02_b200 as zq
 
         self.zq, self.w, self.dtype, self.hadamard = zq, w, dtype, hadamard
+        self.per_kv = per_kv and dtype != "bf16"
         q, k, v = workloads.make_inputs(w, seed=w.seed + seed_offset)
         self.host = [t.pin_memory() for t in (q, k, v)]
         dev = torch.device("cuda")
@@ -211,8 +215,21 @@ class Step:
             self.qc = torch.empty(self.q32.shape, dtype=f8, device=dev)
             self.kc = torch.empty(self.k32.shape, dtype=f8, device=dev)
             self.vc = torch.empty(self.v32.shape, dtype=f8, device=dev)
-            self.ds = torch.zeros(3, dtype=torch.float32, device=dev)
-            self.ws = torch.empty(3, zq.zq_quantize_workspace_bytes(), dtype=torch.uint8, device=dev)
+            if self.per_kv:
+                # one scale per (batch, kv head); the query heads of a kv
+                # head share its scale
+                g = Hq // Hkv
+                self.dsq = torch.zeros((B, Hkv), dtype=torch.float32, device=dev)
+                self.dsk = torch.zeros((B, Hkv), dtype=torch.float32, device=dev)
+                self.dsv = torch.zeros((B, Hkv), dtype=torch.float32, device=dev)
+                nb = max(zq.zq_quantize_grouped_workspace_bytes(B, Hq, g),
+                         zq.zq_quantize_grouped_workspace_bytes(B, Hkv, 1))
+                self.ws = torch.empty(3, nb, dtype=torch.uint8, device=dev)
+                self.group_q = g
+            else:
+                self.ds = torch.zeros(3, dtype=torch.float32, device=dev)
+                self.dsq, self.dsk, self.dsv = self.ds[0:1], self.ds[1:2], self.ds[2:3]
+                self.ws = torch.empty(3, zq.zq_quantize_workspace_bytes(), dtype=torch.uint8, device=dev)
         self.mode = zq.ZQ_SOFTMAX_EXACT if dtype == "exact" else zq.ZQ_SOFTMAX_LEANP
         self.T = T
         self.ev = []
@@ -228,13 +245,21 @@ class Step:
             zq.attn_fwd(self.qb, self.kb, self.vb, out=self.out, lse=self.lse)
         else:
             zq.attn_fwd(self.qc, self.kc, self.vc, out=self.out, lse=self.lse,
-                        q_descale=self.ds[0:1], k_descale=self.ds[1:2], v_descale=self.ds[2:3],
+                        q_descale=self.dsq, k_descale=self.dsk, v_descale=self.dsv,
                         softmax_mode=self.mode, block_scale=True, headroom_T=self.T)
         if ev is not None:
             ev[1].record()
 
     def quantize(self):
         zq = self.zq
+        if self.per_kv:
+            zq.quantize_fp8_grouped(self.q32, self.group_q, hadamard=self.hadamard, out=self.qc,
+                                    descale=self.dsq, workspace=self.ws[0])
+            zq.quantize_fp8_grouped(self.k32, 1, hadamard=self.hadamard, out=self.kc, descale=self.dsk,
+                                    workspace=self.ws[1])
+            zq.quantize_fp8_grouped(self.v32, 1, hadamard=False, out=self.vc, descale=self.dsv,
+                                    workspace=self.ws[2])
+            return
         zq.quantize_fp8(self.q32, hadamard=self.hadamard, out=self.qc, descale=self.ds[0:1], workspace=self.ws[0])
         zq.quantize_fp8(self.k32, hadamard=self.hadamard, out=self.kc, descale=self.ds[1:2], workspace=self.ws[1])
         zq.quantize_fp8(self.v32, hadamard=False, out=self.vc, descale=self.ds[2:3], workspace=self.ws[2])
@@ -281,7 +306,7 @@ def time_steps(fn, steps, warmup, world):
     return max_over_ranks(ms, world)
 
 
-def _oracle_inputs(w, dtype, hadamard):
+def _oracle_inputs(w, dtype, hadamard, per_kv=False):
     """The kernel's inputs for `w` as fp64 arrays (FP8: quantised and decoded,
     as the kernel sees them)."""
     import oracle
@@ -290,6 +315,11 @@ def _oracle_inputs(w, dtype, hadamard):
     if dtype == "bf16":
         return tuple(torch.from_numpy(t).to(torch.bfloat16).double().numpy() for t in (q, k, v))
     deq = []
+    if per_kv:
+        for t, g, rot in ((q, w.Hq // w.Hkv, hadamard), (k, 1, hadamard), (v, 1, False)):
+            c, d = oracle.quantize_fp8_grouped(t, heads_per_scale=g, hadamard=rot)
+            deq.append(oracle.dequant_grouped(c, d))
+        return tuple(deq)
     for t, rot in ((q, hadamard), (k, hadamard), (v, False)):
         c, d = oracle.quantize_fp8(t, hadamard=rot)
         deq.append(oracle.dequant_e4m3(c, float(d)))
@@ -310,12 +340,12 @@ def _oracle_rows(w, dtype, qd, kd, vd, rows):
     return float(np.sum(2.0 * (w.dqk + w.dv) * (i + 1)))
 
 
-def cpu_oracle_rate(w, dtype, seconds, hadamard=False):
+def cpu_oracle_rate(w, dtype, seconds, hadamard=False, per_kv=False):
     """Time the oracle on host cores over a bounded row sample of `w`.
     Returns (TFLOP/s, cores, sample description)."""
     import oracle
 
-    qd, kd, vd = _oracle_inputs(w, dtype, hadamard)
+    qd, kd, vd = _oracle_inputs(w, dtype, hadamard, per_kv)
     rng = np.random.default_rng(0)
     done_rows, flops, elapsed = 0, 0.0, 0.0
     batch = 64
@@ -333,13 +363,13 @@ def cpu_oracle_rate(w, dtype, seconds, hadamard=False):
     return flops / elapsed / 1e12, oracle.num_threads(), desc
 
 
-def oracle_steps(w, dtype, steps, warmup, rows_per_step, hadamard=False):
+def oracle_steps(w, dtype, steps, warmup, rows_per_step, hadamard=False, per_kv=False):
     """The reference arm: `warmup` untimed and `steps` timed oracle steps,
     each over `rows_per_step` query rows drawn uniformly (seeded) from the
     workload.  Returns (TFLOP/s, ms per step, cores, sample description)."""
     import oracle
 
-    qd, kd, vd = _oracle_inputs(w, dtype, hadamard)
+    qd, kd, vd = _oracle_inputs(w, dtype, hadamard, per_kv)
     rng = np.random.default_rng(1)
     for _ in range(warmup):
         _oracle_rows(w, dtype, qd, kd, vd, rng.integers(0, w.B * w.Hq * w.S, size=rows_per_step))
@@ -355,10 +385,17 @@ def oracle_steps(w, dtype, steps, warmup, rows_per_step, hadamard=False):
     return flops / elapsed / 1e12, elapsed / max(steps, 1) * 1e3, oracle.num_threads(), desc
 
 
+def _variant_suffix(args) -> str:
+    suf = "_hadamard" if args.hadamard else ""
+    if args.dtype != "bf16" and getattr(args, "descale", "tensor") == "kv":
+        suf += "_kvscale"
+    return suf
+
+
 def run_ours(args, rank, world, w):
     import bf16_causal_prefill_02_b200 as zq  # noqa: F401  (fails loudly without the .so)
 
-    step = Step(w, args.dtype, args.hadamard, seed_offset=rank, T=args.T)
+    step = Step(w, args.dtype, args.hadamard, seed_offset=rank, T=args.T, per_kv=args.descale == "kv")
     flops = w.causal_flops()
     sampler = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
     # warm-up + attention-only event timing for the roofline
@@ -421,7 +458,7 @@ def run_ours(args, rank, world, w):
     kind = "bf16" if args.dtype == "bf16" else "fp8"
     peak, peak_src = tensor_peak(kind)
     achieved = flops / (attn_ms * 1e-3) / 1e12
-    tkey = "%s_%s_S%d" % (w.name.split("_S")[0], args.dtype, w.S)
+    tkey = "%s_%s_S%d%s" % (w.name.split("_S")[0], args.dtype, w.S, _variant_suffix(args))
     traffic = load_traffic(tkey)
     res = {
         "metric": "causal prefill attention TFLOP/s (FP8, BF16) at S=16K/32K; % of B200 tensor peak",
@@ -429,7 +466,7 @@ def run_ours(args, rank, world, w):
         "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None,
         "dtype": "fp8_e4m3" if kind == "fp8" else "bf16", "data": "synthetic",
-        "config": {"workload": "%s_%s%s" % (w.name, args.dtype, "_hadamard" if args.hadamard else ""),
+        "config": {"workload": "%s_%s%s" % (w.name, args.dtype, _variant_suffix(args)),
                    "B": w.B, "S": w.S, "Hq": w.Hq, "Hkv": w.Hkv, "d_qk": w.dqk, "d_v": w.dv,
                    "causal": True, "softmax": args.dtype,
                    "block_scale": kind == "fp8", "headroom_T": args.T if kind == "fp8" else None,
@@ -460,14 +497,15 @@ def main():
         if rank == 0:
             # each step a bounded sample: about 0.1-0.3 s of oracle work at 32K
             rows = max(32, min(1024, int(256 * 32768 / max(w.S, 1))))
-            tf, ms, cores, desc = oracle_steps(w, args.dtype, args.steps, args.warmup, rows, args.hadamard)
+            tf, ms, cores, desc = oracle_steps(w, args.dtype, args.steps, args.warmup, rows, args.hadamard,
+                                                args.descale == "kv")
             line = {"impl": "reference", "metric": "causal prefill attention TFLOP/s (FP8, BF16) at "
                     "S=16K/32K; % of B200 tensor peak", "value": tf, "unit": "TFLOP/s",
                     "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
                     "warmup": args.warmup, "ms_per_step": round(ms, 3),
                     "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                     "dtype": "f64", "data": "synthetic",
-                    "config": {"workload": "%s_%s%s" % (w.name, args.dtype, "_hadamard" if args.hadamard else ""),
+                    "config": {"workload": "%s_%s%s" % (w.name, args.dtype, _variant_suffix(args)),
                                "B": w.B, "S": w.S, "Hq": w.Hq, "Hkv": w.Hkv, "d_qk": w.dqk, "d_v": w.dv,
                                "causal": True, "softmax": args.dtype},
                     "cpu_baseline": {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
@@ -479,7 +517,8 @@ def main():
     rank, world, local = dist_setup(args.gpus)
     res = run_ours(args, rank, world, w)
     if rank == 0 and not args.no_cpu:
-        tf, cores, desc = cpu_oracle_rate(w, args.dtype, args.cpu_seconds, args.hadamard)
+        tf, cores, desc = cpu_oracle_rate(w, args.dtype, args.cpu_seconds, args.hadamard,
+                                             args.descale == "kv")
         res["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                                "sample": desc}
     if rank == 0:
