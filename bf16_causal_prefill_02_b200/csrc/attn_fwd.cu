@@ -15,14 +15,20 @@
 //        TL;DR (causal prefill, FP8 e4m3 and BF16, d 128 and MLA 192/128) and
 //        "How ZYFA works" (scaling by powers of 2 before rounding).
 //
-// One CTA computes one 128-row query tile of one (batch, head).  Warp roles:
+// A unit is one 128-row query tile of one (batch, head).  With more than 64
+// query tiles per head every CTA runs one unit (grid = units); shorter
+// sequences run persistent CTAs (grid = min(units, SMs)) that take units in
+// a zigzag order and carry their barrier phases from unit to unit.  Warp
+// roles:
 //   warps 0-7  softmax + epilogue.  TMEM lane quarter q (query rows
 //              32q..32q+31) belongs to warps q and q+4, 16 rows each; inside
 //              a warp, threads t and t+16 share a row, thread t taking keys
 //              0-63 of every tile and thread t+16 keys 64-127 (one 64-key
 //              scale block each; 16x32bx2 TMEM accesses)
-//   warp 8     TMA producer (Q per unit, then K and V tiles through two
-//              NS-stage rings that refill independently)
+//   warp 8     TMA producer: Q per unit, then K and V tiles through an
+//              NS-stage ring (K and V of a stage land together), or, with
+//              2 stages (BF16 MLA), through separate K and V rings that
+//              refill independently
 //   warp 9     TMEM allocator and tcgen05 issuer (the whole warp runs the
 //              loop, one elected lane issues)
 // Tensor memory (512 columns x 128 lanes, fp32 words):
