@@ -49,6 +49,13 @@ class zq_attn_args(ctypes.Structure):
     ]
 
 
+class zq_attn_plan(ctypes.Structure):
+    _fields_ = [
+        ("n_units", ctypes.c_int64), ("grid", ctypes.c_int64), ("persistent", ctypes.c_int),
+        ("head_group", ctypes.c_int), ("smem_bytes", ctypes.c_int), ("threads", ctypes.c_int),
+    ]
+
+
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(
@@ -62,6 +69,9 @@ def _load():
     lib.zq_attn_fwd.restype = i32
     lib.zq_attn_fwd_ex.argtypes = [ctypes.POINTER(zq_attn_args), P]
     lib.zq_attn_fwd_ex.restype = i32
+    lib.zq_attn_plan_launch.argtypes = [ctypes.POINTER(zq_attn_args), i32, ctypes.POINTER(zq_attn_plan),
+                                        P, P, P, P, P]
+    lib.zq_attn_plan_launch.restype = i32
     lib.zq_attn_fwd_debug.argtypes = [ctypes.POINTER(zq_attn_args), P, i32, i32, i32, P]
     lib.zq_attn_fwd_debug.restype = i32
     lib.zq_quantize_fp8.argtypes = [P, i32, i64, i32, i32, P, P, P, P]
@@ -104,6 +114,34 @@ def zq_attn_fwd(q, k, v, out, lse, B, Sq, Sk, Hq, Hkv, d_qk, d_v, softmax_scale,
 
 def zq_attn_fwd_ex(args: zq_attn_args, stream) -> int:
     return _lib.zq_attn_fwd_ex(ctypes.byref(args), stream)
+
+
+def zq_attn_plan_launch(args: zq_attn_args, num_sms, plan: zq_attn_plan, unit_tile=None, unit_bh=None,
+                        unit_nkv=None, unit_cta=None, unit_round=None) -> int:
+    """Host-only: the launch shape and per-unit schedule zq_attn_fwd_ex would
+    use.  The unit_* arguments are host addresses of int32 arrays (or None)."""
+    return _lib.zq_attn_plan_launch(ctypes.byref(args), num_sms, ctypes.byref(plan), unit_tile, unit_bh,
+                                    unit_nkv, unit_cta, unit_round)
+
+
+def attn_plan(B, Sq, Sk, Hq, Hkv, d_qk=128, d_v=128, dtype=ZQ_DTYPE_FP8_E4M3, causal=True, num_sms=148):
+    """Schedule of an attention call on the host: (plan, units) with units a
+    dict of numpy int32 arrays tile, bh, n_kv, cta, round indexed by unit."""
+    import numpy as np
+
+    a = zq_attn_args()
+    fake = 1 << 20  # 16-byte aligned; the planner never dereferences it
+    a.q = a.k = a.v = a.out = fake
+    a.B, a.Sq, a.Sk, a.Hq, a.Hkv, a.d_qk, a.d_v = B, Sq, Sk, Hq, Hkv, d_qk, d_v
+    a.causal, a.dtype = int(bool(causal)), dtype
+    a.softmax_mode, a.block_scale, a.headroom_T = ZQ_SOFTMAX_LEANP, 1, 8
+    plan = zq_attn_plan()
+    _check(zq_attn_plan_launch(a, num_sms, plan), "zq_attn_plan_launch")
+    n = int(plan.n_units)
+    arrs = {k: np.full(n, -1, dtype=np.int32) for k in ("tile", "bh", "n_kv", "cta", "round")}
+    _check(zq_attn_plan_launch(a, num_sms, plan, *(arrs[k].ctypes.data for k in ("tile", "bh", "n_kv", "cta", "round"))),
+           "zq_attn_plan_launch")
+    return plan, arrs
 
 
 def zq_attn_fwd_debug(args: zq_attn_args, dbg, dbg_bh, dbg_qtile, flags, stream) -> int:

@@ -50,12 +50,12 @@
 
 #include <cstdint>
 
+#include "schedule.h"
 #include "sm100_ptx.cuh"
 #include "zq_internal.h"
 
 namespace zq {
 
-constexpr int kTile = 128;
 constexpr int kSoftmaxThreads = 256;
 constexpr int kThreads = kSoftmaxThreads + 64;
 constexpr int kWarpProducer = 8, kWarpMma = 9;
@@ -220,30 +220,6 @@ __device__ __forceinline__ uint64_t clk64() {
   return t;
 }
 
-// One work unit: a 128-row query tile t of flat head bh = batch * Hq + head.
-// Units are numbered in groups of head_group consecutive heads; inside a
-// group, longest causal rows first, interleaved across the group's heads.
-struct Unit {
-  int t, bh, b, h, g, q0, n_kv, min_lim;
-};
-__device__ __forceinline__ Unit unit_of(const AttnParams& p, int u) {
-  Unit w;
-  const int GH = p.head_group;
-  const int gi = u / (GH * p.n_qtiles), gr = u % (GH * p.n_qtiles);
-  w.t = p.n_qtiles - 1 - gr / GH;
-  w.bh = gi * GH + gr % GH;
-  w.b = w.bh / p.Hq;
-  w.h = w.bh % p.Hq;
-  w.g = w.h / (p.Hq / p.Hkv);
-  w.q0 = w.t * kTile;
-  const int q1 = min(w.q0 + kTile - 1, p.Sq - 1);
-  const int shift = p.Sk - p.Sq;
-  const int max_key = p.causal ? min(q1 + shift, p.Sk - 1) : p.Sk - 1;
-  w.n_kv = max_key < 0 ? 0 : max_key / kTile + 1;
-  w.min_lim = p.causal ? min(w.q0 + shift, p.Sk - 1) : p.Sk - 1;
-  return w;
-}
-
 // PERSIST = 0: one unit per CTA (the grid has one CTA per unit).
 template <int DT, int DQK, int DV, int MODE, int BS, int DBG, int PERSIST>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -293,14 +269,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
 
   const int n_units = p.n_qtiles * p.B * p.Hq;
-  // The k-th unit of this CTA: rounds of gridDim.x units, walked forwards in
-  // even rounds and backwards in odd ones, so that under longest-rows-first
-  // numbering every CTA pairs long units with short ones (a plain stride
-  // would hand CTA 0 about twice the work of the last CTA).  Strictly
-  // increasing in k.
-  auto unit_at = [&](int k) -> int {
-    return k * (int)gridDim.x + ((k & 1) ? (int)gridDim.x - 1 - (int)blockIdx.x : (int)blockIdx.x);
-  };
+  // the k-th unit of this CTA (zigzag rounds; schedule.h)
+  auto unit_at = [&](int k) -> int { return zq::unit_at(k, (int)gridDim.x, (int)blockIdx.x); };
   const int shift = p.Sk - p.Sq;
   // debug dumps and the trace exist only in the DBG instantiation
   auto traced_unit = [&](const Unit& w) { return DBG && p.dbg != nullptr && w.t == p.dbg_t && w.bh == p.dbg_bh; };
@@ -964,22 +934,17 @@ static cudaError_t launch_variant(const AttnLaunch& a, cudaStream_t st) {
   const long long n_units = (long long)p.n_qtiles * p.B * p.Hq;
   if (n_units <= 0) return cudaSuccess;
   if (n_units > 0x7fffffffLL) return cudaErrorInvalidValue;
-  // Short sequences (at most 64 query tiles) run persistent: one CTA per SM
-  // (all of TMEM), each walking its share of the units (see unit_at in the
-  // kernel), so a unit's loads and first QK overlap the previous unit's tail.
-  // Longer ones launch a CTA per unit from a one-unit instantiation: the
-  // hardware scheduler then balances units of very different lengths better
-  // than the static share, and the per-unit setup is a small part of a long
-  // unit.
-  long long nblocks = n_units;
-  const bool persist = p.n_qtiles <= 64;
+  // persistent CTAs (one per SM) for short sequences, else one CTA per
+  // unit from the one-unit instantiation (schedule.h)
+  const bool persist = use_persistent(p.n_qtiles);
+  int sms = 0;
   if (persist) {
-    int dev = 0, sms = 0;
+    int dev = 0;
     cudaError_t e0 = cudaGetDevice(&dev);
     if (e0 == cudaSuccess) e0 = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e0 != cudaSuccess) return e0;
-    if (sms > 0 && sms < nblocks) nblocks = sms;
   }
+  const long long nblocks = grid_size(p.n_qtiles, n_units, sms);
   auto kern = p.dbg ? (persist ? attn_fwd_kernel<DT, DQK, DV, MODE, BS, 1, 1> : attn_fwd_kernel<DT, DQK, DV, MODE, BS, 1, 0>)
                     : (persist ? attn_fwd_kernel<DT, DQK, DV, MODE, BS, 0, 1> : attn_fwd_kernel<DT, DQK, DV, MODE, BS, 0, 0>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM);
@@ -987,6 +952,13 @@ static cudaError_t launch_variant(const AttnLaunch& a, cudaStream_t st) {
   kern<<<(unsigned)nblocks, kThreads, G::SMEM, st>>>(mQ, mQ2, mK, mK2, mV, p);
   return cudaGetLastError();
 }
+
+int attn_smem_bytes(int dtype, int dqk) {
+  if (dtype == 0) return dqk == 128 ? Geo<0, 128, 128>::SMEM : Geo<0, 192, 128>::SMEM;
+  return dqk == 128 ? Geo<1, 128, 128>::SMEM : Geo<1, 192, 128>::SMEM;
+}
+
+int attn_threads() { return kThreads; }
 
 cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t st) {
   if (a.dtype == 0) {

@@ -9,6 +9,7 @@
 
 #include "zattn.h"
 
+#include "schedule.h"
 #include "zq_internal.h"
 
 namespace {
@@ -52,9 +53,11 @@ int validate_attn(const zq_attn_args* a) {
       return ZQ_ERR_UNSUPPORTED;
   }
   if (!(std::isfinite(a->softmax_scale))) return ZQ_ERR_SHAPE;
-  // grid = n_qtiles * B * Hq blocks; TMA element counts and strides
+  // units = n_qtiles * B * Hq stay in int range, with room above the last
+  // unit for the persistent CTAs' zigzag walk (it computes indices up to
+  // two rounds of CTAs past the last unit); TMA element counts and strides
   const int64_t ntiles = (a->Sq + 127) / 128;
-  if (ntiles * a->B * (int64_t)a->Hq > 0x7FFFFFFFll) return ZQ_ERR_SHAPE;
+  if (ntiles * a->B * (int64_t)a->Hq > 0x7FFF0000ll) return ZQ_ERR_SHAPE;
   const int es = a->dtype == ZQ_DTYPE_BF16 ? 2 : 1;
   const int64_t qbytes = (int64_t)a->B * a->Sq * a->Hq * a->d_qk * es;
   const int64_t kbytes = (int64_t)a->B * a->Sk * a->Hkv * a->d_qk * es;
@@ -85,12 +88,8 @@ const char* zq_status_string(int s) {
   }
 }
 
-static int attn_impl(const zq_attn_args* a, void* dbg, int dbg_bh, int dbg_t, int dbg_flags,
-                     void* stream) {
-  int rc = validate_attn(a);
-  if (rc != ZQ_OK) return rc;
-  rc = check_device(nullptr);
-  if (rc != ZQ_OK) return rc;
+// Launch description of a validated call (no device access).
+static zq::AttnLaunch make_launch(const zq_attn_args* a) {
   zq::AttnLaunch L;
   L.q = a->q;
   L.k = a->k;
@@ -113,25 +112,28 @@ static int attn_impl(const zq_attn_args* a, void* dbg, int dbg_bh, int dbg_t, in
   L.p.Sk = a->Sk;
   L.p.Hq = a->Hq;
   L.p.Hkv = a->Hkv;
-  L.p.n_qtiles = (a->Sq + 127) / 128;
-  {
-    // Group 4 heads (one K/V head under 4:1 GQA) when the K/V of all heads
-    // is well past what the 126 MB L2 keeps around (96 MB): blocks then
-    // stream shared K/V tiles.
-    // Smaller problems keep longest-rows-first over every head, which
-    // balances the tail better.
-    const int bh = a->B * a->Hq;
-    const double es = a->dtype == ZQ_DTYPE_FP8_E4M3 ? 1.0 : 2.0;
-    const double kv_bytes = (double)a->B * a->Hkv * a->Sk * (a->d_qk + a->d_v) * es;
-    int gh = bh;
-    if (kv_bytes > 96.0 * 1024 * 1024) gh = bh % 4 == 0 ? 4 : (bh % 2 == 0 ? 2 : 1);
-    L.p.head_group = gh;
-  }
+  L.p.n_qtiles = (a->Sq + zq::kTile - 1) / zq::kTile;
+  L.p.head_group = zq::choose_head_group(a->B, a->Hq, a->Hkv, a->Sk, a->d_qk, a->d_v,
+                                         a->dtype == ZQ_DTYPE_FP8_E4M3 ? 1 : 2);
   L.p.causal = a->causal ? 1 : 0;
   L.p.headroom_T = a->dtype == ZQ_DTYPE_FP8_E4M3 ? a->headroom_T : 8;
   L.p.softmax_scale =
       a->softmax_scale > 0.0f ? a->softmax_scale : (float)(1.0 / std::sqrt((double)a->d_qk));
   L.p.timeout_ns = kTimeoutNs;
+  L.p.dbg = nullptr;
+  L.p.dbg_bh = 0;
+  L.p.dbg_t = 0;
+  L.p.dbg_flags = 0;
+  return L;
+}
+
+static int attn_impl(const zq_attn_args* a, void* dbg, int dbg_bh, int dbg_t, int dbg_flags,
+                     void* stream) {
+  int rc = validate_attn(a);
+  if (rc != ZQ_OK) return rc;
+  rc = check_device(nullptr);
+  if (rc != ZQ_OK) return rc;
+  zq::AttnLaunch L = make_launch(a);
   L.p.dbg = dbg;
   L.p.dbg_bh = dbg_bh;
   L.p.dbg_t = dbg_t;
@@ -142,6 +144,47 @@ static int attn_impl(const zq_attn_args* a, void* dbg, int dbg_bh, int dbg_t, in
 
 int zq_attn_fwd_ex(const zq_attn_args* a, void* stream) {
   return attn_impl(a, nullptr, 0, 0, 0, stream);
+}
+
+int zq_attn_plan_launch(const zq_attn_args* a, int num_sms, zq_attn_plan* plan,
+                        int32_t* unit_tile, int32_t* unit_bh, int32_t* unit_nkv,
+                        int32_t* unit_cta, int32_t* unit_round) {
+  if (!plan) return ZQ_ERR_NULL;
+  int rc = validate_attn(a);
+  if (rc != ZQ_OK) return rc;
+  if (num_sms <= 0) {
+    rc = check_device(&num_sms);
+    if (rc != ZQ_OK) return rc;
+  }
+  const zq::AttnLaunch L = make_launch(a);
+  const zq::AttnParams& p = L.p;
+  const long long n_units = (long long)p.n_qtiles * p.B * p.Hq;
+  const long long grid = zq::grid_size(p.n_qtiles, n_units, num_sms);
+  plan->n_units = n_units;
+  plan->grid = grid;
+  plan->persistent = zq::use_persistent(p.n_qtiles) ? 1 : 0;
+  plan->head_group = p.head_group;
+  plan->smem_bytes = zq::attn_smem_bytes(a->dtype, a->d_qk);
+  plan->threads = zq::attn_threads();
+  if (!unit_tile && !unit_bh && !unit_nkv && !unit_cta && !unit_round) return ZQ_OK;
+  for (long long u = 0; u < n_units; ++u) {
+    const zq::Unit w = zq::unit_of(p, (int)u);
+    if (unit_tile) unit_tile[u] = w.t;
+    if (unit_bh) unit_bh[u] = w.bh;
+    if (unit_nkv) unit_nkv[u] = w.n_kv;
+  }
+  if (unit_cta || unit_round) {
+    // walk every CTA's sequence exactly as the kernel does
+    for (long long c = 0; c < grid; ++c) {
+      for (int k = 0;; ++k) {
+        const long long u = zq::unit_at(k, (int)grid, (int)c);
+        if (u >= n_units || (k > 0 && !plan->persistent)) break;
+        if (unit_cta) unit_cta[u] = (int32_t)c;
+        if (unit_round) unit_round[u] = k;
+      }
+    }
+  }
+  return ZQ_OK;
 }
 
 int zq_attn_fwd_debug(const zq_attn_args* a, void* dbg, int dbg_bh, int dbg_qtile, int flags,

@@ -51,6 +51,9 @@ struct AttnLaunch {
 };
 
 cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t st);
+// dynamic shared memory and threads of one attention CTA (host side)
+int attn_smem_bytes(int dtype, int dqk);
+int attn_threads();
 // hadamard: 0 none, 1 H128 on every 128-slice (d % 128 == 0), 2 the d = 192
 // rotation (H128 on channels 0..127, sqrt2 * H64 on 128..191)
 cudaError_t launch_quantize(const void* x, int x_bf16, int64_t n, int hadamard, void* out,

@@ -143,6 +143,46 @@ typedef struct zq_attn_args {
  * range (they are ignored, not checked, for bf16). */
 ZQ_API int zq_attn_fwd_ex(const zq_attn_args* args, void* stream);
 
+/* Launch shape of one attention call, from zq_attn_plan_launch. */
+typedef struct zq_attn_plan {
+  int64_t n_units;  /* work units: ceil(Sq / 128) query tiles x B x Hq        */
+  int64_t grid;     /* CTAs launched                                          */
+  int persistent;   /* 1: each CTA walks several units (Sq <= 64 x 128 rows)  */
+  int head_group;   /* flat heads whose tiles are interleaved in unit order  */
+  int smem_bytes;   /* dynamic shared memory per CTA                          */
+  int threads;      /* threads per CTA                                        */
+} zq_attn_plan;
+
+/*
+ * zq_attn_plan_launch -- the schedule zq_attn_fwd_ex would launch for `args`,
+ * computed on the host (host code only; nothing is launched or read from
+ * the device).
+ * [P3 TL;DR: causal prefill -- a query tile visits only key tiles holding a
+ *  key visible to one of its rows; GQA maps query head h to kv head
+ *  h / (Hq / Hkv).]
+ *
+ *   args      validated exactly as by zq_attn_fwd_ex (same errors); the
+ *             device pointers in it are not dereferenced.
+ *   num_sms   SMs to plan for; <= 0 asks the current device (which must
+ *             then be sm_100, else ZQ_ERR_ARCH / ZQ_ERR_CUDA).
+ *   plan      receives the launch shape.
+ *   unit_tile, unit_bh, unit_nkv, unit_cta, unit_round: optional HOST
+ *             arrays of plan->n_units int32 each (NULL to skip; call once
+ *             with all NULL to learn n_units).  Entry u describes work unit
+ *             u: its query tile t (rows 128t..128t+127), its flat head
+ *             b * Hq + h, the number of key tiles it visits (tiles
+ *             0..n_kv-1), the CTA that runs it and its position in that
+ *             CTA's sequence.  Units are numbered in groups of head_group
+ *             heads, longest rows first inside a group; a persistent CTA c
+ *             of G runs, in round k, unit k*G + c (k even) or
+ *             k*G + G-1-c (k odd).
+ * Errors: ZQ_ERR_NULL (plan NULL, or as zq_attn_fwd_ex), ZQ_ERR_SHAPE,
+ *   ZQ_ERR_UNSUPPORTED, ZQ_ERR_ALIGN, ZQ_ERR_ARCH, ZQ_ERR_CUDA.
+ */
+ZQ_API int zq_attn_plan_launch(const zq_attn_args* args, int num_sms, zq_attn_plan* plan,
+                               int32_t* unit_tile, int32_t* unit_bh, int32_t* unit_nkv,
+                               int32_t* unit_cta, int32_t* unit_round);
+
 /* zq_attn_fwd_debug -- zq_attn_fwd_ex that also dumps, for the query tile
  * dbg_qtile (rows 128*dbg_qtile..) of flat head dbg_bh = batch*Hq + head,
  * the first 128x128 score tile before masking and the
