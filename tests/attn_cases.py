@@ -72,22 +72,33 @@ class Case:
         self.vd = oracle.dequant_e4m3(self.cv, float(self.dsv))
 
     # ------------------------------------------------------------ CUDA path
-    def run_gpu(self, debug=None, status=None, out=None, lse=None, debug_at=(0, 0), debug_flags=0):
+    def runner(self):
+        """A function that launches the CUDA path on inputs uploaded once."""
         import bf16_causal_prefill_02_b200 as zq
 
         dev = "cuda"
         if not self.fp8:
             q, k, v = (t.to(dev) for t in (self.qb, self.kb, self.vb))
-            return zq.attn_fwd(q, k, v, causal=self.causal, debug=debug, debug_at=debug_at, status=status,
-                               out=out, lse=lse, debug_flags=debug_flags)
+
+            def run(debug=None, status=None, out=None, lse=None, debug_at=(0, 0), debug_flags=0):
+                return zq.attn_fwd(q, k, v, causal=self.causal, debug=debug, debug_at=debug_at, status=status,
+                                   out=out, lse=lse, debug_flags=debug_flags)
+            return run
         q, k, v = (torch.from_numpy(c).to(dev).view(torch.float8_e4m3fn) for c in (self.cq, self.ck, self.cv))
         dq, dk, dv = (torch.tensor(np.asarray(d, dtype=np.float32).reshape(-1), device=dev)
                       for d in (self.dsq, self.dsk, self.dsv))
         mode = zq.ZQ_SOFTMAX_EXACT if self.dtype == "exact" else zq.ZQ_SOFTMAX_LEANP
-        return zq.attn_fwd(q, k, v, causal=self.causal, q_descale=dq, k_descale=dk, v_descale=dv,
-                           softmax_mode=mode, block_scale=self.block_scale, headroom_T=self.T,
-                           debug=debug, debug_at=debug_at, status=status, out=out, lse=lse,
-                           debug_flags=debug_flags)
+
+        def run(debug=None, status=None, out=None, lse=None, debug_at=(0, 0), debug_flags=0):
+            return zq.attn_fwd(q, k, v, causal=self.causal, q_descale=dq, k_descale=dk, v_descale=dv,
+                               softmax_mode=mode, block_scale=self.block_scale, headroom_T=self.T,
+                               debug=debug, debug_at=debug_at, status=status, out=out, lse=lse,
+                               debug_flags=debug_flags)
+        return run
+
+    def run_gpu(self, debug=None, status=None, out=None, lse=None, debug_at=(0, 0), debug_flags=0):
+        return self.runner()(debug=debug, status=status, out=out, lse=lse, debug_at=debug_at,
+                             debug_flags=debug_flags)
 
     # --------------------------------------------------------------- oracle
     def r1(self, rows=None):

@@ -206,6 +206,22 @@ def test_bitwise_deterministic(dtype):
         assert torch.equal(l.view(torch.int32), l0.view(torch.int32))
 
 
+@pytest.mark.parametrize("dtype", DTYPES)
+def test_bitwise_deterministic_7200_launches_tiny(dtype):
+    # the pages report bitwise identical outputs over 7,200 launches ([P1]
+    # paragraph 2; [P3] "How accurate"); the same count on the tiny workload
+    w = workloads.get("tiny")
+    c = Case(w.B, w.S, w.S, w.Hq, w.Hkv, w.dqk, w.dv, dtype=dtype, inputs=workloads.make_inputs(w))
+    run = c.runner()
+    o0, l0 = run()
+    o, l = torch.empty_like(o0), torch.empty_like(l0)
+    differ = torch.zeros((), dtype=torch.int64, device=o0.device)
+    for _ in range(7200):
+        run(out=o, lse=l)
+        differ += (o.view(torch.int16) != o0.view(torch.int16)).sum() + (l.view(torch.int32) != l0.view(torch.int32)).sum()
+    assert int(differ.item()) == 0
+
+
 @pytest.mark.parametrize("dtype", ["bf16", "leanp"])
 def test_timeout_path_reports_status_and_context_survives(dtype):
     # The MMA issuer withholds all work (test hook): every other role's
