@@ -1,12 +1,13 @@
 """Benchmark: causal prefill attention TFLOP/s on B200 (FP8 e4m3 / BF16).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
-                    [--dtype leanp|exact|bf16] [--impl reference] [--sweep]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--S S]
+                    [--dtype leanp|exact|bf16] [--hadamard] [--descale tensor|kv]
+                    [--T T] [--impl reference] [--sweep]
 
 A step is one pass of the whole hot path over one batch of synthetic input:
-for FP8, the per-tensor quantisation of Q, K and V (fp32 -> e4m3, three
-quantiser calls) followed by the attention kernel; for BF16 the attention
-kernel alone.  The headline workload is the Gaussian peak-sweep point at
+for FP8, the quantisation of Q, K and V (fp32 -> e4m3, three quantiser calls;
+one scale per tensor, or with --descale kv one per (batch, kv head))
+followed by the attention kernel; for BF16 the attention kernel alone.  The headline workload is the Gaussian peak-sweep point at
 S = 32768 (B=1, Hq=Hkv=32, d=128), FP8 with Lean P and per-64-key block
 scaling -- the configuration the pages quote their best FP8 number on.
 
@@ -470,7 +471,9 @@ def run_ours(args, rank, world, w):
                    "B": w.B, "S": w.S, "Hq": w.Hq, "Hkv": w.Hkv, "d_qk": w.dqk, "d_v": w.dv,
                    "causal": True, "softmax": args.dtype,
                    "block_scale": kind == "fp8", "headroom_T": args.T if kind == "fp8" else None,
-                   "step": ("quantise Q,K,V (fp32->e4m3) + attention" if kind == "fp8" else "attention"),
+                   "step": (("quantise Q,K,V (fp32->e4m3, %s scales) + attention" %
+                             ("per-(batch, kv head)" if step.per_kv else "per-tensor"))
+                            if kind == "fp8" else "attention"),
                    "l2": "inputs larger than L2 (%.0f MB fp32 Q/K/V), no flush" %
                          (3 * w.B * w.S * w.Hq * w.dqk * 4 / 1e6),
                    "parallelism": "dp%d (independent batches, no collective)" % world},
