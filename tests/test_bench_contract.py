@@ -40,3 +40,12 @@ def test_reference_arm_other_ranks_are_silent():
     lines = _run(["--impl", "reference", "--workload", "tiny", "--steps", "2", "--warmup", "1"],
                  {"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
     assert lines == []
+
+
+def test_reference_arm_per_kv_head_scales():
+    lines = _run(["--impl", "reference", "--workload", "tiny", "--steps", "2", "--warmup", "1",
+                  "--descale", "kv", "--hadamard"])
+    assert len(lines) == 1
+    r = lines[0]
+    assert r["config"]["workload"] == "tiny_leanp_hadamard_kvscale"
+    assert r["value"] > 0 and r["cpu_baseline"]["kind"] == "oracle"
