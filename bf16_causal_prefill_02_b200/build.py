@@ -21,7 +21,7 @@ CSRC = os.path.join(HERE, "csrc")
 OUT = os.path.join(HERE, "libzattn.so")
 BUILD_DIR = os.path.join(ROOT, "_build")
 SOURCES = ["zattn_api.cu", "quantize.cu", "attn_fwd.cu"]
-HEADERS = ["sm100_ptx.cuh", "zq_internal.h"]
+HEADERS = ["sm100_ptx.cuh", "zq_internal.h", "schedule.h"]
 
 
 def nvcc() -> str:
