@@ -182,13 +182,43 @@ def tensor_peak(kind: str):
     return base, "%s bf16 sustained" % src
 
 
+def kernel_sources_digest(read=None) -> str:
+    """sha256 over the attention kernel's sources: attn_fwd.cu and every
+    header beside it, by name in sorted order.  `read(name)` returns a
+    file's bytes (default: the files in csrc)."""
+    import hashlib
+
+    csrc = os.path.join(ROOT, "bf16_causal_prefill_02_b200", "csrc")
+    if read is None:
+        names = sorted(n for n in os.listdir(csrc) if n == "attn_fwd.cu" or n.endswith((".h", ".cuh")))
+
+        def read(n):
+            with open(os.path.join(csrc, n), "rb") as f:
+                return f.read()
+    else:
+        names = sorted(read(None))
+    h = hashlib.sha256()
+    for n in names:
+        h.update(n.encode() + b"\0" + read(n) + b"\0")
+    return h.hexdigest()
+
+
 def load_traffic(key: str):
+    """DRAM bytes per attention launch from profiles/traffic.json, or None.
+    The counters hold only for the kernel they were taken on: when the
+    kernel's sources no longer hash to the digest recorded with them, the
+    figure is returned as stale (second value) and the first is None."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
-        return None
+        return None, None
     with open(path) as f:
         d = json.load(f)
-    return d.get(key)
+    val = d.get(key)
+    if val is None:
+        return None, None
+    if d.get("_kernel_sources_sha256") != kernel_sources_digest():
+        return None, val
+    return val, None
 
 
 # --------------------------------------------------------------- our arm
@@ -460,7 +490,7 @@ def run_ours(args, rank, world, w):
     peak, peak_src = tensor_peak(kind)
     achieved = flops / (attn_ms * 1e-3) / 1e12
     tkey = "%s_%s_S%d%s" % (w.name.split("_S")[0], args.dtype, w.S, _variant_suffix(args))
-    traffic = load_traffic(tkey)
+    traffic, traffic_stale = load_traffic(tkey)
     res = {
         "metric": "causal prefill attention TFLOP/s (FP8, BF16) at S=16K/32K; % of B200 tensor peak",
         "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -480,6 +510,8 @@ def run_ours(args, rank, world, w):
         "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel", "achieved": round(achieved, 1),
                      "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                      "peak_source": peak_src, "traffic": traffic,
+                     "traffic_stale": traffic_stale,
+                     "kernel_sources_sha256": kernel_sources_digest(),
                      "frac_of_datasheet_dense": round(achieved / DATASHEET_DENSE_TFLOPS[kind], 4),
                      "attn_ms": round(attn_ms, 4)},
         "clocks": clocks,

@@ -49,3 +49,26 @@ def test_reference_arm_per_kv_head_scales():
     r = lines[0]
     assert r["config"]["workload"] == "tiny_leanp_hadamard_kvscale"
     assert r["value"] > 0 and r["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_traffic_is_reported_only_for_the_kernel_it_was_taken_on():
+    sys.path.insert(0, ROOT)
+    import bench
+
+    files = {"attn_fwd.cu": b"kernel", "sm100_ptx.cuh": b"ptx", "zq_internal.h": b"params"}
+
+    def read(n):
+        return list(files) if n is None else files[n]
+    d0 = bench.kernel_sources_digest(read)
+    assert d0 == bench.kernel_sources_digest(read)
+    files["attn_fwd.cu"] = b"kernel, changed"
+    assert bench.kernel_sources_digest(read) != d0
+    # the recorded figures carry the digest of the sources they were taken on
+    val, stale = bench.load_traffic("gauss_leanp_S32768")
+    with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+        rec = json.load(f)
+    if rec["_kernel_sources_sha256"] == bench.kernel_sources_digest():
+        assert val == rec["gauss_leanp_S32768"] and stale is None
+    else:
+        assert val is None and stale == rec["gauss_leanp_S32768"]
+    assert bench.load_traffic("no_such_workload") == (None, None)
