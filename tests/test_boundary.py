@@ -160,3 +160,16 @@ def test_no_cpu_fallback_without_library(tmp_path, monkeypatch):
     mod = importlib.util.module_from_spec(spec)
     with pytest.raises(ImportError):
         spec.loader.exec_module(mod)
+
+
+def test_torch_helpers_reject_host_tensors():
+    # the helpers never fall back to the CPU: host tensors are refused
+    import torch
+
+    x = torch.zeros((1, 4, 2, 128))
+    with pytest.raises(ValueError):
+        zq.quantize_fp8(x)
+    with pytest.raises(ValueError):
+        zq.quantize_fp8_grouped(x, heads_per_scale=1)
+    with pytest.raises(ValueError):
+        zq.attn_fwd(x.bfloat16(), x.bfloat16(), x.bfloat16())
