@@ -6,9 +6,11 @@ only used for device memory and streams.  There is no CPU fallback: if the
 shared library is missing, importing this package raises.
 
 Low-level names mirror the C ABI (``zq_attn_fwd``, ``zq_attn_fwd_ex``,
-``zq_quantize_fp8``, ...) and take raw integers (device addresses, sizes, a
-stream handle).  The torch-level helpers ``attn_fwd``, ``quantize_fp8`` and
-``flash_attn_func`` marshal tensors into those calls.
+``zq_quantize_fp8``, ``zq_quantize_fp8_grouped``, ``zq_attn_plan_launch``,
+...) and take raw integers (device addresses, sizes, a stream handle).  The
+torch-level helpers ``attn_fwd``, ``quantize_fp8``, ``quantize_fp8_grouped``
+and ``flash_attn_func`` marshal tensors into those calls; ``attn_plan``
+returns the schedule of a call (host only).
 """
 from __future__ import annotations
 
