@@ -48,6 +48,7 @@
 #include <cuda_runtime.h>
 #include <cuda.h>
 
+#include <atomic>
 #include <cstdint>
 
 #include "schedule.h"
@@ -882,17 +883,22 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// The driver's encoder, looked up once and cached.  Callers on several host
+// threads may race to the first lookup: the cache is atomic, and every
+// thread stores the same pointer.  A failed lookup is retried on the next
+// call.
 static EncodeTiledFn get_encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
-            cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      return nullptr;
-    fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  }
+  static std::atomic<EncodeTiledFn> cache{nullptr};
+  EncodeTiledFn fn = cache.load(std::memory_order_acquire);
+  if (fn) return fn;
+  void* ptr = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
+          cudaSuccess ||
+      q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  cache.store(fn, std::memory_order_release);
   return fn;
 }
 
