@@ -14,7 +14,10 @@
  *   - Pointers named q, k, v, out, lse, x, x_fp8, descale, workspace and
  *     status are DEVICE pointers on the current CUDA device; the caller owns
  *     all of them.  The library allocates nothing and keeps no state between
- *     calls (it is safe to call from several host threads).
+ *     calls besides two lookup caches (the driver's tensor-map encoder, and
+ *     per device the address of the fixed scratch array of
+ *     zq_quantize_fp8_noalloc), both filled atomically; it is safe to call
+ *     from several host threads.
  *   - `stream` is a cudaStream_t passed as void*; NULL is the legacy default
  *     stream.  Every call is asynchronous on that stream and never
  *     synchronises.
