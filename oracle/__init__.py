@@ -21,6 +21,7 @@ Functions (all fp64 unless stated):
                         per (batch, kv head), the flash_attn_func FP8 layout
   dequant_grouped       codes times the per-(batch, head group) descale
   e4m3_decode/encode    OCP e4m3fn codec
+  leanp_code            the Lean P byte of a log2-domain value (R2's rounding)
   brute_attn            dense numpy softmax for tiny inputs (a cross-check)
 
 Every function here is pinned by ``tests/test_oracle.py`` against something
@@ -61,6 +62,10 @@ def _L():
         P = ctypes.c_void_p
         i32, i64, f64 = ctypes.c_int, ctypes.c_int64, ctypes.c_double
         lib.zo_num_threads.restype = i32
+        lib.zo_set_num_threads.argtypes = [i32]
+        lib.zo_set_num_threads.restype = i32
+        lib.zo_leanp_code.argtypes = [f64]
+        lib.zo_leanp_code.restype = i32
         lib.zo_e4m3_decode.argtypes = [ctypes.c_uint8]
         lib.zo_e4m3_decode.restype = f64
         lib.zo_e4m3_encode_rne_sat.argtypes = [f64]
@@ -85,6 +90,20 @@ def _ptr(a):
 
 def num_threads() -> int:
     return int(_L().zo_num_threads())
+
+
+def set_num_threads(n: int) -> int:
+    """Thread count of the oracle's parallel loops (timing only; results do
+    not depend on it).  Returns the count in effect."""
+    return int(_L().zo_set_num_threads(int(n)))
+
+
+def leanp_code(z) -> np.ndarray:
+    """Lean P byte of each log2-domain value z = y - e: 8z rounded half to
+    even, plus 56, clamped to [0, 126] (the function R2 uses)."""
+    z = np.asarray(z, dtype=np.float64)
+    f = _L().zo_leanp_code
+    return np.array([f(float(t)) for t in z.ravel()], dtype=np.int64).reshape(z.shape)
 
 
 # ----------------------------------------------------------------- codec

@@ -28,6 +28,7 @@
  *        rotation uses it, scaled by fl32(sqrt 2), on channels 128..191.
  *   zo_quantize_fp8     per-tensor amax quantiser (R3).
  *   zo_attn_ref         exact fp64 softmax(QK^T*scale + causal mask)V (R1).
+ *   zo_leanp_code       Lean P byte for a log2-domain value (used by R2).
  *   zo_attn_fp8_emul    scalar emulation of the FP8 P path: per-(row,64-key
  *        block) power-of-2 scaling, exact-exp2 or Lean P rounding, division
  *        by the sum of the rounded probabilities (R2).
@@ -44,6 +45,19 @@ int zo_num_threads(void) {
 #ifdef _OPENMP
   return omp_get_max_threads();
 #else
+  return 1;
+#endif
+}
+
+/* Thread count for the parallel loops that follow (n <= 0: leave as is).
+ * Returns the count now in effect.  Only timing uses it (the single-thread
+ * rate of the CPU baseline); results do not depend on it. */
+int zo_set_num_threads(int n) {
+#ifdef _OPENMP
+  if (n > 0) omp_set_num_threads(n);
+  return omp_get_max_threads();
+#else
+  (void)n;
   return 1;
 #endif
 }
@@ -281,7 +295,7 @@ int zo_attn_ref(const double* q, const double* k, const double* v, int B, int Sq
  * 56 = 7*8 gives the pattern of 2^z; P2 "Perche l'FP8 non basta da solo":
  * 2^x from a multiply-add and an integer conversion).  Rounding of 8*z is
  * half-to-even; the code is clamped to the finite range [0, 126]. */
-static int leanp_code(double z) {
+int zo_leanp_code(double z) {
   double t = 8.0 * z;
   double r = nearbyint(t); /* default rounding mode: ties to even */
   double c = r + 56.0;
@@ -372,7 +386,7 @@ int zo_attn_fp8_emul(const double* q, const double* k, const double* v, int B, i
         if (mode == 0)
           p = zo_e4m3_decode(zo_e4m3_encode_rne_sat(exp2(z)));
         else if (mode == 1)
-          p = zo_e4m3_decode((uint8_t)leanp_code(z));
+          p = zo_e4m3_decode((uint8_t)zo_leanp_code(z));
         else
           p = exp2(z);
         pt[c] = p;

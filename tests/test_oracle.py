@@ -284,9 +284,118 @@ def test_leanp_closed_form_and_mitchell_bounds():
         ratio = pb[normal] / np.exp2(z[normal])
         assert np.all(ratio >= 2.0 ** (-1 / 16) * 0.999999)
         assert np.all(ratio <= 1.0615 * 2.0 ** (1 / 16))
-    # at integer log2 values the code is 8t+56 and the value is exactly 2^t
-    codes = oracle.e4m3_encode(np.exp2(np.arange(-6, 9, dtype=np.float64)))
-    assert list(codes) == [8 * t + 56 for t in range(-6, 9)]
+    # at integer log2 values the Lean P code is 8t+56 and its value exactly 2^t
+    t = np.arange(-6, 9)
+    codes = oracle.leanp_code(t.astype(np.float64))
+    assert list(codes) == [8 * x + 56 for x in t]
+    assert np.array_equal(_torch_e4m3_value(codes), np.exp2(t.astype(np.float64)))
+
+
+def _torch_e4m3_value(codes):
+    """Value of e4m3fn bytes as torch decodes them (independent of the oracle)."""
+    c = torch.from_numpy(np.asarray(codes, dtype=np.uint8).copy())
+    return c.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+def test_leanp_code_integers_ties_and_clamp():
+    # [P1] paragraph 3: an e4m3 byte read as an integer grows by 8 per
+    # doubling, so 8z + 56 is the byte of 2^z; the reading rounds 8z half to
+    # even and clamps to the finite codes [0, 126].
+    # Integers: code 8t + 56; t = -7 is the clamp edge (code 0).
+    t = np.arange(-7, 9)
+    assert list(oracle.leanp_code(t.astype(np.float64))) == [8 * x + 56 for x in t]
+    # Exact half codes (8z = k + 1/2) land on the even neighbour: never the
+    # odd one that half-away-from-zero rounding gives for k >= 0 (and k < -1)
+    k = np.arange(-55, 70)
+    z = (k + 0.5) / 8.0
+    c = oracle.leanp_code(z)
+    assert np.all(c % 2 == 0)
+    assert np.all(np.abs(c - (8.0 * z + 56.0)) == 0.5)
+    assert list(oracle.leanp_code(np.array([0.0625, -0.0625, 0.1875, -0.1875]))) == [56, 56, 58, 54]
+    # Clamp at zero: 8z = -55.5 is a tie whose even neighbour -56 gives code 0;
+    # anything below stays 0; just above the tie the code is 1
+    assert list(oracle.leanp_code(np.array([-6.9375, -7.0, -9.5, -300.0]))) == [0, 0, 0, 0]
+    assert oracle.leanp_code(np.array([-6.9375 + 1e-9]))[0] == 1
+    # Clamp at the top: never the NaN byte 127
+    assert list(oracle.leanp_code(np.array([8.75, 9.0, 50.0]))) == [126, 126, 126]
+    assert oracle.leanp_code(np.array([8.5625]))[0] == 124  # 8z = 68.5 -> 68
+    # Monotone in z
+    g = np.linspace(-8.0, 9.0, 20001)
+    assert np.all(np.diff(oracle.leanp_code(g)) >= 0)
+
+
+def _exact_dot(y, scale=1.0):
+    """A dot product d with fl(fl(scale * d) * log2 e) == y exactly (the
+    emulation's score arithmetic), searched over neighbouring doubles."""
+    L = 1.4426950408889634
+    d0 = y / (scale * L)
+    a = b = d0
+    for _ in range(400):
+        for d in (a, b):
+            if (scale * d) * L == y:
+                return d
+        a, b = np.nextafter(a, np.inf), np.nextafter(b, -np.inf)
+    raise AssertionError("no exact input for %r" % y)
+
+
+def test_emul_leanp_ties_and_clamp_inside_a_row():
+    # One non-causal row, d = 1, scale 1: the scores are the dot products
+    # times log2 e, built so that y is exact.  Block max 4.6 gives
+    # e = ceil(4.6) - 8 = -3; the other keys sit at exact half codes of
+    # z = y - e and at the clamp.
+    zs = [0.0625, -0.0625, 0.1875, -0.1875, 0.3125, -6.9375]
+    want = [56, 56, 58, 54, 58, 0]
+    ys = [4.6] + [-3.0 + z for z in zs]
+    dots = [_exact_dot(y) for y in ys]
+    Sk = len(dots)
+    q = np.ones((1, 1, 1, 1))
+    k = np.array(dots, dtype=np.float64).reshape(1, Sk, 1, 1)
+    v = np.ones((1, Sk, 1, 1))
+    _, _, p = oracle.attn_fp8_emul(q, k, v, scale=1.0, causal=False, mode=oracle.MODE_LEANP, T=8,
+                                   want_p=True)
+    assert np.array_equal(p[1:], _torch_e4m3_value(want))
+    assert 2.0 ** 7 < p[0] <= 2.0 ** 8
+
+
+def _running_mode_row():
+    """One query row over three 128-key tiles (d = 1, scale 1): tile 0 peaks
+    at 2.3, tile 1 stays below that (its peak is key 10 of the tile, 1.7),
+    tile 2 rises to 4.6.  Key 10 of each tile has the same score 1.7."""
+    rng = np.random.default_rng(5)
+    L = 1.4426950408889634
+    y = np.concatenate([rng.uniform(-3.0, 2.0, 128), rng.uniform(-3.0, 1.0, 128), rng.uniform(-3.0, 4.0, 128)])
+    y[50], y[128 + 70], y[256 + 90] = 2.3, 1.1, 4.6
+    y[[10, 138, 266]] = 1.7
+    dots = y / L
+    q = np.ones((1, 1, 1, 1))
+    k = dots.reshape(1, 384, 1, 1)
+    v = rng.standard_normal((1, 384, 1, 4))
+    return q, k, v
+
+
+@pytest.mark.parametrize("mode", [oracle.MODE_EXACT, oracle.MODE_LEANP])
+def test_emul_running_mode_exponent_per_tile(mode):
+    # block_scale = 0: one exponent per 128-key tile, e_t = ceil(running max
+    # of y over tiles 0..t) - T, shared by both 64-key blocks.  With T = 8:
+    # tile 0: e = ceil(2.3) - 8 = -5 (largest p~ in (2^7, 2^8]); tile 1 keeps
+    # e = -5 (its own peak 1.7 is below the running max, so its largest p~ is
+    # below 2^7, and key 138 equals key 10); tile 2: e = ceil(4.6) - 8 = -3
+    # (largest p~ back in (2^7, 2^8], key 266 is key 10 divided by exactly 4).
+    q, k, v = _running_mode_row()
+    _, _, p = oracle.attn_fp8_emul(q, k, v, scale=1.0, causal=False, mode=mode, block_scale=False, T=8,
+                                   want_p=True)
+    t0, t1, t2 = p[:128], p[128:256], p[256:]
+    assert 2.0 ** 7 < t0.max() <= 2.0 ** 8
+    assert t1.max() <= 2.0 ** 7
+    assert 2.0 ** 7 < t2.max() <= 2.0 ** 8
+    assert p[138] == p[10] and p[10] > 0
+    assert p[266] * 4.0 == p[10]
+    # block-local scaling on the same row: every 64-key block peaks in (2^7, 2^8]
+    _, _, pb = oracle.attn_fp8_emul(q, k, v, scale=1.0, causal=False, mode=mode, block_scale=True, T=8,
+                                    want_p=True)
+    for j0 in range(0, 384, 64):
+        assert 2.0 ** 7 < pb[j0:j0 + 64].max() <= 2.0 ** 8
+    assert pb[138] == 2.0 * pb[10]  # tile 1's first block: e = ceil(1.7) - 8 = -6
 
 
 def test_exact_mode_p_is_rounded_exp2():
