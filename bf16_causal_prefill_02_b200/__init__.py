@@ -20,8 +20,7 @@ import os
 import re
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-# ZQ_LIB_PATH selects another build of the same library (for comparing builds).
-LIB_PATH = os.environ.get("ZQ_LIB_PATH") or os.path.join(HERE, "libzattn.so")
+LIB_PATH = os.path.join(HERE, "libzattn.so")
 HEADER_PATH = os.path.join(os.path.dirname(HERE), "include", "zattn.h")
 
 ZQ_DTYPE_BF16, ZQ_DTYPE_FP8_E4M3 = 0, 1
@@ -224,6 +223,28 @@ def _is_fp8(t) -> bool:
     return t.dtype in (torch.float8_e4m3fn, torch.uint8)
 
 
+def _check_buffer(name, t, shape, dtype):
+    """A caller-supplied output or side buffer: contiguous, exact shape and dtype."""
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError("%s must have shape %s, got %s" % (name, tuple(shape), tuple(t.shape)))
+    if t.dtype != dtype:
+        raise ValueError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+
+
+def _check_same_cuda_device(dev, named):
+    """Every given tensor lives on CUDA device `dev` (no host pointers reach
+    the library, and no tensor of another GPU)."""
+    for name, t in named:
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError("%s must be a CUDA tensor" % name)
+        if t.device != dev:
+            raise ValueError("%s is on %s, expected %s" % (name, t.device, dev))
+
+
 def quantize_fp8(x, hadamard: bool = False, out=None, descale=None, workspace=None, stream=None):
     """Per-tensor e4m3 quantisation of a CUDA tensor (fp32 or bf16, last dim d).
 
@@ -237,13 +258,24 @@ def quantize_fp8(x, hadamard: bool = False, out=None, descale=None, workspace=No
         xd = ZQ_X_BF16
     else:
         raise TypeError("quantize_fp8 takes float32 or bfloat16")
+    if x.dim() == 0:
+        raise ValueError("x needs a last (channel) dimension")
     d = x.shape[-1]
     if out is None:
         out = torch.empty(x.shape, dtype=torch.float8_e4m3fn, device=x.device)
+    elif out.dtype not in (torch.float8_e4m3fn, torch.uint8):
+        raise ValueError("out must be float8_e4m3fn or uint8")
+    else:
+        _check_buffer("out", out, x.shape, out.dtype)
     if descale is None:
         descale = torch.empty(1, dtype=torch.float32, device=x.device)
+    else:
+        _check_buffer("descale", descale, (1,), torch.float32)
     if workspace is None:
         workspace = torch.empty(zq_quantize_workspace_bytes(), dtype=torch.uint8, device=x.device)
+    elif workspace.numel() * workspace.element_size() < zq_quantize_workspace_bytes() or not workspace.is_contiguous():
+        raise ValueError("workspace must be contiguous and hold zq_quantize_workspace_bytes() bytes")
+    _check_same_cuda_device(x.device, [("out", out), ("descale", descale), ("workspace", workspace)])
     _check(zq_quantize_fp8(x.data_ptr(), xd, x.numel() // d, d, int(bool(hadamard)), out.data_ptr(),
                            descale.data_ptr(), workspace.data_ptr(), _stream(stream)), "zq_quantize_fp8")
     return out, descale
@@ -272,11 +304,20 @@ def quantize_fp8_grouped(x, heads_per_scale=1, hadamard: bool = False, out=None,
         raise ValueError("heads_per_scale must divide the head count")
     if out is None:
         out = torch.empty(x.shape, dtype=torch.float8_e4m3fn, device=x.device)
+    elif out.dtype not in (torch.float8_e4m3fn, torch.uint8):
+        raise ValueError("out must be float8_e4m3fn or uint8")
+    else:
+        _check_buffer("out", out, x.shape, out.dtype)
     if descale is None:
         descale = torch.empty((B, H // g), dtype=torch.float32, device=x.device)
+    elif descale.numel() != B * (H // g) or descale.dtype != torch.float32 or not descale.is_contiguous():
+        raise ValueError("descale must be a contiguous float32 tensor of B * H / heads_per_scale values")
+    nbytes = zq_quantize_grouped_workspace_bytes(B, H, g)
     if workspace is None:
-        nbytes = zq_quantize_grouped_workspace_bytes(B, H, g)
         workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=x.device)
+    elif workspace.numel() * workspace.element_size() < nbytes or not workspace.is_contiguous():
+        raise ValueError("workspace must be contiguous and hold zq_quantize_grouped_workspace_bytes() bytes")
+    _check_same_cuda_device(x.device, [("out", out), ("descale", descale), ("workspace", workspace)])
     _check(zq_quantize_fp8_grouped(x.data_ptr(), xd, B, S, H, d, g, int(bool(hadamard)), out.data_ptr(),
                                    descale.data_ptr(), workspace.data_ptr(), _stream(stream)),
            "zq_quantize_fp8_grouped")
@@ -306,9 +347,11 @@ def attn_fwd(q, k, v, out=None, lse=None, softmax_scale=None, causal=True, q_des
     quantize_fp8_grouped returns them).
     Returns (out bf16 (B,Sq,Hq,d_v), lse fp32 (B,Hq,Sq) or None)."""
     torch = _torch()
-    for t in (q, k, v):
-        if not t.is_cuda or not t.is_contiguous():
-            raise ValueError("q, k, v must be contiguous CUDA tensors")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.dim() != 4:
+            raise ValueError("%s must be 4-D (batch, seq, heads, dim), got %d-D" % (name, t.dim()))
+        if not t.is_contiguous():
+            raise ValueError("%s must be contiguous" % name)
     if _is_fp8(q) and _is_fp8(k) and _is_fp8(v):
         dtype = ZQ_DTYPE_FP8_E4M3
     elif q.dtype == k.dtype == v.dtype == torch.bfloat16:
@@ -317,10 +360,34 @@ def attn_fwd(q, k, v, out=None, lse=None, softmax_scale=None, causal=True, q_des
         raise TypeError("q, k, v must all be bfloat16 or all FP8 e4m3")
     B, Sq, Hq, dqk = q.shape
     Sk, Hkv, dv = k.shape[1], k.shape[2], v.shape[3]
+    # the kernel addresses k and v with q's batch and k's sequence, heads and
+    # width: every pair must agree, or it would read past an allocation
+    if k.shape[0] != B or v.shape[0] != B:
+        raise ValueError("q, k, v must have the same batch size, got %d, %d, %d" % (B, k.shape[0], v.shape[0]))
+    if k.shape[3] != dqk:
+        raise ValueError("k must have q's head dim %d, got %d" % (dqk, k.shape[3]))
+    if v.shape[1] != Sk or v.shape[2] != Hkv:
+        raise ValueError("v must have k's sequence length and head count (%d, %d), got (%d, %d)"
+                         % (Sk, Hkv, v.shape[1], v.shape[2]))
     if out is None:
         out = torch.empty((B, Sq, Hq, dv), dtype=torch.bfloat16, device=q.device)
+    else:
+        _check_buffer("out", out, (B, Sq, Hq, dv), torch.bfloat16)
     if lse is None and return_lse:
         lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    elif lse is not None:
+        _check_buffer("lse", lse, (B, Hq, Sq), torch.float32)
+    descales = (("q_descale", q_descale), ("k_descale", k_descale), ("v_descale", v_descale))
+    if dtype == ZQ_DTYPE_FP8_E4M3:
+        for name, t in descales:
+            if t is not None and (t.dtype != torch.float32 or not t.is_contiguous()):
+                raise ValueError("%s must be a contiguous float32 tensor" % name)
+    if status is not None and (status.dtype != torch.int32 or status.numel() < 1):
+        raise ValueError("status must be an int32 tensor with at least one element")
+    if debug is not None and debug.numel() * debug.element_size() < ZQ_DEBUG_BYTES:
+        raise ValueError("debug must hold ZQ_DEBUG_BYTES bytes")
+    _check_same_cuda_device(q.device, [("q", q), ("k", k), ("v", v), ("out", out), ("lse", lse), ("status", status),
+                                       ("debug", debug)] + (list(descales) if dtype == ZQ_DTYPE_FP8_E4M3 else []))
     a = zq_attn_args()
     a.q, a.k, a.v, a.out, a.lse = q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), _ptr(lse)
     a.B, a.Sq, a.Sk, a.Hq, a.Hkv, a.d_qk, a.d_v = B, Sq, Sk, Hq, Hkv, dqk, dv

@@ -264,3 +264,39 @@ def test_full_size_sampled_rows(name, dtype, had):
     rows = workloads.sample_rows(w.B, w.Hq, w.S, every=every).numpy()
     res = check_against_oracle(c, rows=rows)
     print(name, dtype, had, res)
+
+
+@pytest.mark.parametrize("dtype,dqk", [("bf16", 128), ("leanp", 128), ("bf16", 192), ("leanp", 192)])
+def test_plain_c_entry_zq_attn_fwd(dtype, dqk):
+    # The flash_attn_func-style C call itself (not the extended entry):
+    # raw device addresses, sizes and a stream handle through the C ABI.
+    # For FP8 it runs Lean P with block scaling and headroom 8.
+    import bf16_causal_prefill_02_b200 as zq
+
+    B, S, Hq, Hkv = 2, 333, 4, 2
+    c = Case(B, S, S, Hq, Hkv, dqk, 128, dtype=dtype, seed=60 + dqk)
+    dev = "cuda"
+    out = torch.full((B, S, Hq, 128), float("nan"), dtype=torch.bfloat16, device=dev)
+    lse = torch.full((B, Hq, S), float("nan"), dtype=torch.float32, device=dev)
+    if c.fp8:
+        q, k, v = (torch.from_numpy(x).to(dev) for x in (c.cq, c.ck, c.cv))
+        ds = [torch.tensor([float(d)], dtype=torch.float32, device=dev) for d in (c.dsq, c.dsk, c.dsv)]
+        dptr = [d.data_ptr() for d in ds]
+        code = zq.ZQ_DTYPE_FP8_E4M3
+    else:
+        q, k, v = (t.to(dev) for t in (c.qb, c.kb, c.vb))
+        dptr = [None, None, None]
+        code = zq.ZQ_DTYPE_BF16
+    stream = torch.cuda.current_stream().cuda_stream
+    rc = zq.zq_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, S, S,
+                        Hq, Hkv, dqk, 128, 0.0, 1, code, dptr[0], dptr[1], dptr[2], stream)
+    assert rc == zq.ZQ_OK, zq.zq_status_string(rc)
+    torch.cuda.synchronize()
+    check_against_oracle(c, o_gpu=out, lse_gpu=lse)
+    # lse NULL: the output alone, bit-identical to the run with lse
+    out2 = torch.empty_like(out)
+    rc = zq.zq_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out2.data_ptr(), None, B, S, S,
+                        Hq, Hkv, dqk, 128, 0.0, 1, code, dptr[0], dptr[1], dptr[2], stream)
+    assert rc == zq.ZQ_OK
+    torch.cuda.synchronize()
+    assert torch.equal(out2.view(torch.int16), out.view(torch.int16))
