@@ -72,3 +72,21 @@ def test_traffic_is_reported_only_for_the_kernel_it_was_taken_on():
     else:
         assert val is None and stale == rec["gauss_leanp_S32768"]
     assert bench.load_traffic("no_such_workload") == (None, None)
+
+
+def test_reference_arm_config_matches_ours():
+    # both arms describe the workload with the same function, so the driver
+    # sees identical config dicts for the same command line
+    sys.path.insert(0, ROOT)
+    import argparse
+
+    import bench
+    import workloads
+
+    lines = _run(["--impl", "reference", "--workload", "tiny", "--steps", "2", "--warmup", "1"])
+    args = argparse.Namespace(dtype="leanp", hadamard=False, descale="tensor", T=8)
+    ours = bench.config_dict(workloads.get("tiny"), args, 1)
+    assert lines[0]["config"] == ours
+    for key in ("block_scale", "headroom_T", "step", "l2", "parallelism"):
+        assert key in ours
+    assert lines[0]["cpu_baseline"]["cpu_model"]
