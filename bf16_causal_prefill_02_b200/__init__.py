@@ -6,10 +6,11 @@ only used for device memory and streams.  There is no CPU fallback: if the
 shared library is missing, importing this package raises.
 
 Low-level names mirror the C ABI (``zq_attn_fwd``, ``zq_attn_fwd_ex``,
-``zq_quantize_fp8``, ``zq_quantize_fp8_grouped``, ``zq_attn_plan_launch``,
-...) and take raw integers (device addresses, sizes, a stream handle).  The
-torch-level helpers ``attn_fwd``, ``quantize_fp8``, ``quantize_fp8_grouped``
-and ``flash_attn_func`` marshal tensors into those calls; ``attn_plan``
+``zq_quantize_fp8``, ``zq_quantize_fp8_multi``, ``zq_quantize_fp8_grouped``,
+``zq_attn_plan_launch``, ...) and take raw integers (device addresses, sizes,
+a stream handle).  The torch-level helpers ``attn_fwd``, ``quantize_fp8``,
+``quantize_fp8_multi``, ``quantize_fp8_grouped`` and ``flash_attn_func``
+marshal tensors into those calls; ``attn_plan``
 returns the schedule of a call (host only).
 """
 from __future__ import annotations
@@ -50,6 +51,13 @@ class zq_attn_args(ctypes.Structure):
     ]
 
 
+class zq_quant_tensor(ctypes.Structure):
+    _fields_ = [
+        ("x", ctypes.c_void_p), ("x_dtype", ctypes.c_int), ("n_vec", ctypes.c_int64), ("d", ctypes.c_int),
+        ("hadamard", ctypes.c_int), ("x_fp8", ctypes.c_void_p), ("descale", ctypes.c_void_p),
+    ]
+
+
 class zq_attn_plan(ctypes.Structure):
     _fields_ = [
         ("n_units", ctypes.c_int64), ("grid", ctypes.c_int64), ("persistent", ctypes.c_int),
@@ -77,6 +85,10 @@ def _load():
     lib.zq_attn_fwd_debug.restype = i32
     lib.zq_quantize_fp8.argtypes = [P, i32, i64, i32, i32, P, P, P, P]
     lib.zq_quantize_fp8.restype = i32
+    lib.zq_quantize_fp8_multi.argtypes = [ctypes.POINTER(zq_quant_tensor), i32, P, P]
+    lib.zq_quantize_fp8_multi.restype = i32
+    lib.zq_quantize_multi_workspace_bytes.argtypes = []
+    lib.zq_quantize_multi_workspace_bytes.restype = ctypes.c_size_t
     lib.zq_quantize_fp8_noalloc.argtypes = [P, i32, i64, i32, i32, P, P, P]
     lib.zq_quantize_fp8_noalloc.restype = i32
     lib.zq_quantize_fp8_grouped.argtypes = [P, i32, i32, i64, i32, i32, i32, i32, P, P, P, P]
@@ -154,6 +166,15 @@ ZQ_DEBUG_BYTES = 128 * 128 * 4 + 128 * 64 * 4 + 256 * 4 + 512 * 16 * 8
 
 def zq_quantize_fp8(x, x_dtype, n_vec, d, hadamard, x_fp8, descale, workspace, stream) -> int:
     return _lib.zq_quantize_fp8(x, x_dtype, n_vec, d, hadamard, x_fp8, descale, workspace, stream)
+
+
+def zq_quantize_fp8_multi(tensors, count, workspace, stream) -> int:
+    """`tensors`: a ctypes array (or pointer) of zq_quant_tensor."""
+    return _lib.zq_quantize_fp8_multi(tensors, count, workspace, stream)
+
+
+def zq_quantize_multi_workspace_bytes() -> int:
+    return int(_lib.zq_quantize_multi_workspace_bytes())
 
 
 def zq_quantize_fp8_noalloc(x, x_dtype, n_vec, d, hadamard, x_fp8, descale, stream) -> int:
@@ -279,6 +300,58 @@ def quantize_fp8(x, hadamard: bool = False, out=None, descale=None, workspace=No
     _check(zq_quantize_fp8(x.data_ptr(), xd, x.numel() // d, d, int(bool(hadamard)), out.data_ptr(),
                            descale.data_ptr(), workspace.data_ptr(), _stream(stream)), "zq_quantize_fp8")
     return out, descale
+
+
+def quantize_fp8_multi(xs, hadamard=None, outs=None, descales=None, workspace=None, stream=None):
+    """Per-tensor e4m3 quantisation of up to four CUDA tensors in one call
+    (three stream operations in all), e.g. q, k, v with the rotation on q and k.
+
+    hadamard: one flag per tensor (default all False).  Returns (codes list,
+    descales list), each as quantize_fp8 returns them for the tensor alone."""
+    torch = _torch()
+    xs = list(xs)
+    n = len(xs)
+    if not 1 <= n <= 4:
+        raise ValueError("quantize_fp8_multi takes 1 to 4 tensors")
+    hadamard = [False] * n if hadamard is None else [bool(h) for h in hadamard]
+    if len(hadamard) != n:
+        raise ValueError("one hadamard flag per tensor")
+    outs = [None] * n if outs is None else list(outs)
+    descales = [None] * n if descales is None else list(descales)
+    arr = (zq_quant_tensor * n)()
+    for i, x in enumerate(xs):
+        if not x.is_cuda or not x.is_contiguous() or x.dim() == 0:
+            raise ValueError("every tensor must be a contiguous CUDA tensor")
+        if x.dtype == torch.float32:
+            xd = ZQ_X_F32
+        elif x.dtype == torch.bfloat16:
+            xd = ZQ_X_BF16
+        else:
+            raise TypeError("quantize_fp8_multi takes float32 or bfloat16")
+        if x.device != xs[0].device:
+            raise ValueError("all tensors must be on one device")
+        if outs[i] is None:
+            outs[i] = torch.empty(x.shape, dtype=torch.float8_e4m3fn, device=x.device)
+        elif outs[i].dtype not in (torch.float8_e4m3fn, torch.uint8):
+            raise ValueError("out must be float8_e4m3fn or uint8")
+        else:
+            _check_buffer("out", outs[i], x.shape, outs[i].dtype)
+        if descales[i] is None:
+            descales[i] = torch.empty(1, dtype=torch.float32, device=x.device)
+        else:
+            _check_buffer("descale", descales[i], (1,), torch.float32)
+        _check_same_cuda_device(x.device, [("out", outs[i]), ("descale", descales[i])])
+        d = x.shape[-1]
+        arr[i].x, arr[i].x_dtype, arr[i].n_vec, arr[i].d = x.data_ptr(), xd, x.numel() // d, d
+        arr[i].hadamard, arr[i].x_fp8, arr[i].descale = int(hadamard[i]), outs[i].data_ptr(), descales[i].data_ptr()
+    nbytes = zq_quantize_multi_workspace_bytes()
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=xs[0].device)
+    elif workspace.numel() * workspace.element_size() < nbytes or not workspace.is_contiguous():
+        raise ValueError("workspace must be contiguous and hold zq_quantize_multi_workspace_bytes() bytes")
+    _check_same_cuda_device(xs[0].device, [("workspace", workspace)])
+    _check(zq_quantize_fp8_multi(arr, n, workspace.data_ptr(), _stream(stream)), "zq_quantize_fp8_multi")
+    return outs, descales
 
 
 def quantize_fp8_grouped(x, heads_per_scale=1, hadamard: bool = False, out=None, descale=None,

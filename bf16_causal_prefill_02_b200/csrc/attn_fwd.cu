@@ -90,7 +90,7 @@ struct Geo {
   static constexpr int OFF_SF = OFF_ONES + ONES_BYTES;     // FP8: [2 buf] 512 B scale tiles
   static constexpr int SF_BYTES = DT == 1 ? 1024 : 0;
   static constexpr int OFF_BAR = OFF_SF + SF_BYTES;
-  static constexpr int NBAR = 1 + 4 * NS + 2 + 2 + 1 + 2;
+  static constexpr int NBAR = 1 + 4 * NS + 2 + 2 + 1 + 2 + 1;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;  // + alignment slack
   static_assert(SMEM <= 232448, "227 KB of shared memory per CTA");
   static_assert(DV == 128, "the two halves of a row split d_v = 128 in 64 + 64");
@@ -257,6 +257,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // (jt) and of units with work (nq).
   uint64_t* bar_qfree = bar_ofinal + 1;       // [1] last QK of a unit done: Q reusable
   uint64_t* bar_ofree = bar_qfree + 1;        // [1] softmax read O (and RS) of a unit
+  uint64_t* bar_drain = bar_ofree + 1;        // [1] after an abort: the MMA issuer's work landed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + G::NBAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   // FP8 scale factors staged for tcgen05.cp: per S buffer a 32-row x
@@ -293,6 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar_ofinal, 1);
     mbar_init(bar_qfree, 1);
     mbar_init(bar_ofree, kSoftmaxThreads);
+    mbar_init(bar_drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -320,6 +322,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tbase = *tmem_slot;
   const uint64_t lim = p.timeout_ns;
 
+  // producer: the last load armed on each barrier, for the drain after an
+  // abort -- Q loads issued, and the CTA-wide tile index of the last K/V (or
+  // K and V) stage armed
+  int q_loads = 0, x_last = -1, xk_last = -1, xv_last = -1;
+
   auto fail = [&]() {
     *abort_flag = 1;
     if (p.status) atomicExch(p.status, -7 /* ZQ_ERR_TIMEOUT */);
@@ -337,6 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (nq > 0 && !mbar_wait(bar_qfree, (nq - 1) & 1, lim, abort_flag)) { ok = false; break; }
         uint8_t* sq = smem + G::OFF_Q;
         mbar_arrive_expect_tx(bar_q, G::QBYTES);
+        ++q_loads;
 #pragma unroll
         for (int c = 0; c < G::NCH; ++c) {
           const bool narrow = (c == G::NCH - 1) && G::LASTW == 64;
@@ -351,6 +359,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint8_t* sk = smem + G::OFF_K + s * G::KBYTES;
             uint8_t* sv = smem + G::OFF_V + s * G::VBYTES;
             mbar_arrive_expect_tx(bar_kfull + s, G::KBYTES + G::VBYTES);
+            x_last = x;
 #pragma unroll
             for (int c = 0; c < G::NCH; ++c) {
               const bool narrow = (c == G::NCH - 1) && G::LASTW == 64;
@@ -373,6 +382,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (mbar_test_wait(smem_u32(bar_kfree + s), ((x / G::NS) & 1) ^ 1)) {  // first pass: free
                 uint8_t* sk = smem + G::OFF_K + s * G::KBYTES;
                 mbar_arrive_expect_tx(bar_kfull + s, G::KBYTES);
+                xk_last = x;
 #pragma unroll
                 for (int c = 0; c < G::NCH; ++c) {
                   const bool narrow = (c == G::NCH - 1) && G::LASTW == 64;
@@ -388,6 +398,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (mbar_test_wait(smem_u32(bar_vfree + s), ((x / G::NS) & 1) ^ 1)) {
                 uint8_t* sv = smem + G::OFF_V + s * G::VBYTES;
                 mbar_arrive_expect_tx(bar_vfull + s, G::VBYTES);
+                xv_last = x;
 #pragma unroll
                 for (int c = 0; c < G::VCH; ++c)
                   tma_load_4d(sv + c * 16384, &tmV, bar_vfull + s, c * 128 / G::ES, w.g, jv * kTile, w.b);
@@ -836,10 +847,37 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (n_kv > 0) ++nq;
     }  // units
     if (!ok && lane == 0) fail();
+    // no tensor-memory access of this thread is still in flight
+    tmem_ld_wait();
+    tmem_st_wait();
   }
 
   tc_fence_before();
   __syncthreads();
+  if (*abort_flag) {
+    // Some role gave up (a wait ran out): asynchronous work already issued
+    // lands before the CTA frees its tensor memory and exits.  Each waits
+    // again at most the time limit.
+    if (warp == kWarpProducer && lane == 0) {
+      // every TMA load into shared memory: a barrier's last armed phase
+      // completes only once all its bytes arrived (earlier phases of the
+      // same barrier were consumed before it was re-armed)
+      if (q_loads > 0) mbar_wait_bounded(bar_q, (q_loads - 1) & 1, lim);
+      for (int x = max(x_last - G::NS + 1, 0); x <= x_last; ++x)
+        mbar_wait_bounded(bar_kfull + x % G::NS, (x / G::NS) & 1, lim);
+      for (int x = max(xk_last - G::NS + 1, 0); x <= xk_last; ++x)
+        mbar_wait_bounded(bar_kfull + x % G::NS, (x / G::NS) & 1, lim);
+      for (int x = max(xv_last - G::NS + 1, 0); x <= xv_last; ++x)
+        mbar_wait_bounded(bar_vfull + x % G::NS, (x / G::NS) & 1, lim);
+    }
+    if (warp == kWarpMma) {
+      // every MMA and scale copy the issuing lane started
+      if (elect_one()) tc_commit(bar_drain);
+      __syncwarp();
+      mbar_wait_bounded(bar_drain, 0, lim);
+    }
+    __syncthreads();
+  }
   if (warp == kWarpMma) {
     tc_fence_after();
     tmem_dealloc(tbase, kTmemCols);

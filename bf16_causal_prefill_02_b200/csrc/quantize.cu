@@ -427,6 +427,144 @@ cudaError_t launch_quantize(const void* x, int x_bf16, int64_t n, int hadamard, 
 }
 
 // ---------------------------------------------------------------------------
+// Several tensors in one pass pair (Q, K and V of an attention call): one
+// clear of the amax words, one amax launch and one write launch whose grid
+// row blockIdx.y is the tensor.  Each tensor is quantised exactly as by the
+// per-tensor kernels above (same per-thread element walk relative to its own
+// grid, same fp32 operations), so the bytes and descales are identical.
+template <bool BF16IN, bool HAD>
+__device__ __forceinline__ float amax_part(const void* x, int64_t n, int64_t t0, int64_t nthreads, int lane) {
+  float m = 0.0f;
+  for (int64_t i = t0 * 4; i < n; i += nthreads * 4) {
+    float v[4];
+    load4<BF16IN>(x, i, v);
+    if constexpr (HAD) fwht128_warp(v, lane);
+    m = fmaxf(m, fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3]))));
+  }
+  return m;
+}
+
+template <bool BF16IN>
+__device__ __forceinline__ float amax192_part(const void* x, int64_t n_vec, int64_t w0, int64_t nwarps, int lane) {
+  float m = 0.0f;
+  for (int64_t vec = w0; vec < n_vec; vec += nwarps) {
+    float a[4], c[2];
+    load4<BF16IN>(x, vec * 192 + 4 * lane, a);
+    load2<BF16IN>(x, vec * 192 + 128 + 2 * lane, c);
+    fwht128_warp(a, lane);
+    fwht64x2_warp_scaled(c, lane);
+    m = fmaxf(m, fmaxf(fmaxf(fabsf(a[0]), fabsf(a[1])), fmaxf(fabsf(a[2]), fabsf(a[3]))));
+    m = fmaxf(m, fmaxf(fabsf(c[0]), fabsf(c[1])));
+  }
+  return m;
+}
+
+template <bool BF16IN, bool HAD>
+__device__ __forceinline__ void write_part(const void* x, int64_t n, float inv, uint8_t* out, int64_t t0,
+                                           int64_t nthreads, int lane) {
+  for (int64_t i = t0 * 4; i < n; i += nthreads * 4) {
+    float v[4];
+    load4<BF16IN>(x, i, v);
+    if constexpr (HAD) fwht128_warp(v, lane);
+    *reinterpret_cast<uint32_t*>(out + i) = e4m3x4(v, inv);
+  }
+}
+
+template <bool BF16IN>
+__device__ __forceinline__ void write192_part(const void* x, int64_t n_vec, float inv, uint8_t* out, int64_t w0,
+                                              int64_t nwarps, int lane) {
+  for (int64_t vec = w0; vec < n_vec; vec += nwarps) {
+    float a[4], c[2];
+    load4<BF16IN>(x, vec * 192 + 4 * lane, a);
+    load2<BF16IN>(x, vec * 192 + 128 + 2 * lane, c);
+    fwht128_warp(a, lane);
+    fwht64x2_warp_scaled(c, lane);
+    *reinterpret_cast<uint32_t*>(out + vec * 192 + 4 * lane) = e4m3x4(a, inv);
+    const __nv_fp8x2_storage_t t = __nv_cvt_float2_to_fp8x2(
+        make_float2(__fmul_rn(c[0], inv), __fmul_rn(c[1], inv)), __NV_SATFINITE, __NV_E4M3);
+    *reinterpret_cast<uint16_t*>(out + vec * 192 + 128 + 2 * lane) = (uint16_t)t;
+  }
+}
+
+__global__ void __launch_bounds__(256) quant_multi_amax_kernel(QuantItems Q, unsigned* __restrict__ amax_bits) {
+  const QuantItem I = Q.it[blockIdx.y];
+  const int lane = threadIdx.x & 31;
+  // this tensor's own grid: its first `blocks` CTAs of the row
+  const int64_t nb = I.blocks;
+  float m = 0.0f;
+  if ((int64_t)blockIdx.x < nb) {
+    if (I.had == 2) {
+      const int64_t w0 = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+      const int64_t nw = nb * (blockDim.x >> 5);
+      m = I.bf16 ? amax192_part<true>(I.x, I.n / 192, w0, nw, lane) : amax192_part<false>(I.x, I.n / 192, w0, nw, lane);
+    } else {
+      const int64_t t0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+      const int64_t nt = nb * blockDim.x;
+      if (I.bf16)
+        m = I.had ? amax_part<true, true>(I.x, I.n, t0, nt, lane) : amax_part<true, false>(I.x, I.n, t0, nt, lane);
+      else
+        m = I.had ? amax_part<false, true>(I.x, I.n, t0, nt, lane) : amax_part<false, false>(I.x, I.n, t0, nt, lane);
+    }
+  }
+  const float r = block_max_256(m);
+  if (threadIdx.x == 0 && (int64_t)blockIdx.x < nb) atomicMax(amax_bits + blockIdx.y, __float_as_uint(r));
+}
+
+__global__ void __launch_bounds__(256) quant_multi_write_kernel(QuantItems Q, const unsigned* __restrict__ amax_bits) {
+  const QuantItem I = Q.it[blockIdx.y];
+  const int64_t nb = I.blocks;
+  if ((int64_t)blockIdx.x >= nb) return;
+  const int lane = threadIdx.x & 31;
+  const float amax = __uint_as_float(amax_bits[blockIdx.y]);
+  const float inv = amax > 0.0f ? __fdiv_rn(448.0f, amax) : 1.0f;
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    float ds = __fdiv_rn(amax, 448.0f);
+    if (I.had) ds = __fmul_rn(ds, 0.08838834764831845f);  // fl32(2^-3.5)
+    *I.descale = ds;
+  }
+  if (I.had == 2) {
+    const int64_t w0 = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int64_t nw = nb * (blockDim.x >> 5);
+    if (I.bf16) write192_part<true>(I.x, I.n / 192, inv, I.out, w0, nw, lane);
+    else write192_part<false>(I.x, I.n / 192, inv, I.out, w0, nw, lane);
+  } else {
+    const int64_t t0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t nt = nb * blockDim.x;
+    if (I.bf16) {
+      if (I.had) write_part<true, true>(I.x, I.n, inv, I.out, t0, nt, lane);
+      else write_part<true, false>(I.x, I.n, inv, I.out, t0, nt, lane);
+    } else {
+      if (I.had) write_part<false, true>(I.x, I.n, inv, I.out, t0, nt, lane);
+      else write_part<false, false>(I.x, I.n, inv, I.out, t0, nt, lane);
+    }
+  }
+}
+
+// Blocks of one tensor in the per-tensor launcher below (the same count,
+// so that the element walk of every thread is the same).
+static int quant_blocks(int64_t n, int hadamard, int num_sms) {
+  const int threads = 256;
+  const int64_t cap = (int64_t)num_sms * 8;
+  const int64_t want = hadamard == 2 ? (n / 192 + (threads / 32) - 1) / (threads / 32) : (n / 4 + threads - 1) / threads;
+  return (int)(want < cap ? (want > 0 ? want : 1) : cap);
+}
+
+cudaError_t launch_quantize_multi(QuantItems Q, int count, void* workspace, cudaStream_t st, int num_sms) {
+  unsigned* amax = static_cast<unsigned*>(workspace);
+  cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(unsigned) * (size_t)count, st);
+  if (e != cudaSuccess) return e;
+  int gx = 1;
+  for (int t = 0; t < count; ++t) {
+    Q.it[t].blocks = quant_blocks(Q.it[t].n, Q.it[t].had, num_sms);
+    if (Q.it[t].blocks > gx) gx = Q.it[t].blocks;
+  }
+  const dim3 grid(gx, count);
+  quant_multi_amax_kernel<<<grid, 256, 0, st>>>(Q, amax);
+  quant_multi_write_kernel<<<grid, 256, 0, st>>>(Q, amax);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
 // Allocation-free variant.  Some callers cannot hand the library a device
 // workspace: hosts whose device memory is owned by another allocator that
 // offers no scratch API, and latency-critical serving loops that forbid

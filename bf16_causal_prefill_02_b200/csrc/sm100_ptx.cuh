@@ -76,6 +76,19 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
   }
 }
 
+// Wait for a phase without watching the abort flag (the drain after an
+// abort: asynchronous copies and MMAs already issued must land before the
+// CTA frees its tensor memory and exits).  Still bounded by `limit_ns`.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  const uint32_t a = smem_u32(bar);
+  if (mbar_try_wait(a, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t n = 1;; ++n) {
+    if (mbar_try_wait(a, parity)) return true;
+    if ((n & 255u) == 0 && globaltimer_ns() - t0 > limit_ns) return false;
+  }
+}
+
 // True in exactly one lane of the (fully active) warp.
 __device__ __forceinline__ bool elect_one() {
   uint32_t pred = 0;

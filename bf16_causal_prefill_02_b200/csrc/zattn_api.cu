@@ -113,7 +113,7 @@ static zq::AttnLaunch make_launch(const zq_attn_args* a) {
   L.p.Hq = a->Hq;
   L.p.Hkv = a->Hkv;
   L.p.n_qtiles = (a->Sq + zq::kTile - 1) / zq::kTile;
-  L.p.head_group = zq::choose_head_group(a->B, a->Hq, a->Hkv, a->Sk, a->d_qk, a->d_v,
+  L.p.head_group = zq::choose_head_group(a->B, a->Hq, a->Hkv, a->Sq, a->Sk, a->d_qk, a->d_v,
                                          a->dtype == ZQ_DTYPE_FP8_E4M3 ? 1 : 2);
   L.p.causal = a->causal ? 1 : 0;
   L.p.headroom_T = a->dtype == ZQ_DTYPE_FP8_E4M3 ? a->headroom_T : 8;
@@ -242,6 +242,36 @@ int zq_quantize_fp8(const void* x, int x_dtype, int64_t n_vec, int d, int hadama
   cudaError_t e = zq::launch_quantize(x, x_dtype == ZQ_X_BF16, n_vec * (int64_t)d,
                                       hadamard ? (d % 128 == 0 ? 1 : 2) : 0, x_fp8, descale, workspace,
                                       static_cast<cudaStream_t>(stream), sms);
+  return e == cudaSuccess ? ZQ_OK : ZQ_ERR_CUDA;
+}
+
+size_t zq_quantize_multi_workspace_bytes(void) { return 256; }
+
+int zq_quantize_fp8_multi(const zq_quant_tensor* t, int count, void* workspace, void* stream) {
+  if (!t || !workspace) return ZQ_ERR_NULL;
+  if (count < 1 || count > zq::kMaxQuantItems) return ZQ_ERR_SHAPE;
+  zq::QuantItems Q = {};
+  for (int i = 0; i < count; ++i) {
+    const zq_quant_tensor& a = t[i];
+    if (!a.descale) return ZQ_ERR_NULL;
+    if (a.n_vec < 0 || a.d <= 0) return ZQ_ERR_SHAPE;
+    if (a.n_vec > 0 && (!a.x || !a.x_fp8)) return ZQ_ERR_NULL;
+    if (a.x_dtype != ZQ_X_F32 && a.x_dtype != ZQ_X_BF16) return ZQ_ERR_UNSUPPORTED;
+    if (a.d % 8 != 0 || (a.hadamard && a.d % 128 != 0 && a.d != 192)) return ZQ_ERR_UNSUPPORTED;
+    if (a.n_vec > (int64_t)1 << 40 || a.n_vec * (int64_t)a.d > ((int64_t)1 << 40)) return ZQ_ERR_SHAPE;
+    if (!aligned16(a.x) || !aligned16(a.x_fp8)) return ZQ_ERR_ALIGN;
+    Q.it[i].x = a.x;
+    Q.it[i].out = static_cast<uint8_t*>(a.x_fp8);
+    Q.it[i].descale = a.descale;
+    Q.it[i].n = a.n_vec * (int64_t)a.d;
+    Q.it[i].bf16 = a.x_dtype == ZQ_X_BF16 ? 1 : 0;
+    Q.it[i].had = a.hadamard ? (a.d % 128 == 0 ? 1 : 2) : 0;
+  }
+  if (!aligned16(workspace)) return ZQ_ERR_ALIGN;
+  int sms = 0;
+  int rc = check_device(&sms);
+  if (rc != ZQ_OK) return rc;
+  cudaError_t e = zq::launch_quantize_multi(Q, count, workspace, static_cast<cudaStream_t>(stream), sms);
   return e == cudaSuccess ? ZQ_OK : ZQ_ERR_CUDA;
 }
 

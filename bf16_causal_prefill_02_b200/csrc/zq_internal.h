@@ -63,6 +63,21 @@ cudaError_t launch_quantize(const void* x, int x_bf16, int64_t n, int hadamard, 
 cudaError_t launch_quantize_grouped(const void* x, int x_bf16, int B, int64_t S, int H, int d, int g,
                                     int hadamard, void* out, float* descale, void* workspace,
                                     cudaStream_t st, int num_sms);
+// One tensor of a multi-tensor quantiser call: n elements (n % 4 == 0; for
+// had == 2, n % 192 == 0), bf16 input or fp32, had 0 none / 1 H128 / 2 the
+// d = 192 rotation.  `blocks` is filled in by the launcher.
+struct QuantItem {
+  const void* x;
+  uint8_t* out;
+  float* descale;
+  int64_t n;
+  int bf16, had, blocks;
+};
+constexpr int kMaxQuantItems = 4;
+struct QuantItems {
+  QuantItem it[kMaxQuantItems];
+};
+cudaError_t launch_quantize_multi(QuantItems Q, int count, void* workspace, cudaStream_t st, int num_sms);
 void* noalloc_scratch_for_device(int dev);
 cudaError_t launch_exp2_check(const float* x, float* y, int64_t n, int degree, cudaStream_t st);
 size_t noalloc_scratch_capacity();

@@ -236,6 +236,40 @@ ZQ_API int zq_quantize_fp8(const void* x, int x_dtype, int64_t n_vec, int d, int
 ZQ_API size_t zq_quantize_workspace_bytes(void);
 
 /*
+ * zq_quantize_fp8_multi -- zq_quantize_fp8 applied to `count` tensors at
+ * once (1 <= count <= 4; the query, key and value inputs of one attention
+ * call), each with its own scale.  [P2 "Perche l'FP8 non basta da solo": the
+ * inputs are quantised per tensor, with the rotation on Q and K only.]
+ *
+ *   t[i]     one tensor: the arguments of zq_quantize_fp8 (x, x_dtype,
+ *            n_vec, d, hadamard, x_fp8, descale), validated the same way;
+ *            every tensor's bytes and descale equal what zq_quantize_fp8
+ *            writes for it alone.
+ *   workspace  device scratch of zq_quantize_multi_workspace_bytes() bytes,
+ *            16-byte aligned; its contents on entry do not matter and it must
+ *            not be used by another call that runs at the same time.
+ * The call makes three stream operations in all (a clear of `count` words and
+ * two kernels) instead of three per tensor.  Outputs must not overlap inputs
+ * or each other.
+ * Errors: those of zq_quantize_fp8 for any tensor; ZQ_ERR_NULL (t or
+ *   workspace NULL), ZQ_ERR_SHAPE (count outside 1..4).
+ */
+typedef struct zq_quant_tensor {
+  const void* x;
+  int x_dtype;
+  int64_t n_vec;
+  int d;
+  int hadamard;
+  void* x_fp8;
+  float* descale;
+} zq_quant_tensor;
+
+ZQ_API int zq_quantize_fp8_multi(const zq_quant_tensor* t, int count, void* workspace, void* stream);
+
+/* Bytes of device scratch zq_quantize_fp8_multi needs (a small constant). */
+ZQ_API size_t zq_quantize_multi_workspace_bytes(void);
+
+/*
  * zq_quantize_fp8_noalloc -- zq_quantize_fp8 without a workspace argument.
  * (The pages describe no counterpart; this is a library convenience.)
  *
@@ -257,6 +291,10 @@ ZQ_API size_t zq_quantize_workspace_bytes(void);
  * last call's contents (the amax word is cleared at the start of each call),
  * so calls whose work can overlap on the GPU -- on different streams without
  * ordering between them -- race and must not be issued that way.
+ * The cached address belongs to the device's primary context as it was at
+ * the first call: a device reset (cudaDeviceReset) or any other teardown of
+ * that context invalidates it, and calling this entry point on the device
+ * afterwards in the same process is not supported.
  */
 ZQ_API int zq_quantize_fp8_noalloc(const void* x, int x_dtype, int64_t n_vec, int d, int hadamard,
                                    void* x_fp8, float* descale, void* stream);

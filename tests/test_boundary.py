@@ -244,3 +244,36 @@ def test_binding_has_no_library_override():
     src = inspect.getsource(zq)
     assert "os.environ" not in src
     assert zq.LIB_PATH == os.path.join(os.path.dirname(zq.__file__), "libzattn.so")
+
+
+def _qt(**kw):
+    t = zq.zq_quant_tensor()
+    d = dict(x=A, x_dtype=0, n_vec=4, d=128, hadamard=0, x_fp8=A, descale=A)
+    d.update(kw)
+    for k, v in d.items():
+        setattr(t, k, v)
+    return t
+
+
+@pytest.mark.parametrize("items,count,ws,code", [
+    ([{}], 0, A, zq.ZQ_ERR_SHAPE),
+    ([{}] * 5, 5, A, zq.ZQ_ERR_SHAPE),
+    ([{}], 1, None, zq.ZQ_ERR_NULL),
+    ([{}, dict(descale=None)], 2, A, zq.ZQ_ERR_NULL),
+    ([{}, dict(x=None)], 2, A, zq.ZQ_ERR_NULL),
+    ([dict(n_vec=-1)], 1, A, zq.ZQ_ERR_SHAPE),
+    ([{}, {}, dict(d=0)], 3, A, zq.ZQ_ERR_SHAPE),
+    ([dict(x_dtype=2)], 1, A, zq.ZQ_ERR_UNSUPPORTED),
+    ([{}, dict(d=12)], 2, A, zq.ZQ_ERR_UNSUPPORTED),
+    ([dict(d=320, hadamard=1)], 1, A, zq.ZQ_ERR_UNSUPPORTED),
+    ([{}, dict(x=A + 4)], 2, A, zq.ZQ_ERR_ALIGN),
+    ([dict(x_fp8=A + 1)], 1, A, zq.ZQ_ERR_ALIGN),
+    ([{}], 1, A + 8, zq.ZQ_ERR_ALIGN),
+])
+def test_quantize_multi_argument_errors(items, count, ws, code):
+    arr = (zq.zq_quant_tensor * len(items))(*[_qt(**kw) for kw in items])
+    assert zq.zq_quantize_fp8_multi(arr, count, ws, None) == code
+
+
+def test_quantize_multi_workspace_bytes():
+    assert zq.zq_quantize_multi_workspace_bytes() >= 16

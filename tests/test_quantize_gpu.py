@@ -138,3 +138,50 @@ def test_quantize_grouped_empty_sequence():
     codes, ds = zq.quantize_fp8_grouped(torch.zeros((2, 0, 4, 128), device="cuda"), heads_per_scale=2)
     torch.cuda.synchronize()
     assert codes.numel() == 0 and ds.shape == (2, 2) and not ds.cpu().any()
+
+
+@pytest.mark.parametrize("case", [
+    # (shape, src, hadamard) per tensor: Q, K, V of an attention call
+    [((2, 300, 4, 128), "f32", True), ((2, 300, 2, 128), "f32", True), ((2, 300, 2, 128), "f32", False)],
+    [((1, 257, 2, 192), "bf16", True), ((1, 257, 2, 192), "f32", True), ((1, 257, 2, 128), "bf16", False)],
+    [((4096, 32, 128), "f32", False)],
+    [((0, 128), "f32", False), ((5, 8), "f32", False), ((33, 256), "bf16", True), ((1, 192), "f32", True)],
+])
+def test_quantize_multi_bitwise_equals_oracle_per_tensor(case):
+    # one call for several tensors: every tensor's codes and descale are the
+    # oracle's quantiser applied to that tensor alone (mixed dtypes, the
+    # rotation on some, d = 192, an empty tensor)
+    import bf16_causal_prefill_02_b200 as zq
+
+    xs, refs, flags = [], [], []
+    for k, (shape, src, had) in enumerate(case):
+        x = torch.randn(shape, generator=torch.Generator().manual_seed(11 + k)) * (1.0 + 3 * k)
+        if src == "bf16":
+            xb = x.to(torch.bfloat16)
+            refs.append(oracle.quantize_fp8(xb.view(torch.int16).numpy().view(np.uint16), hadamard=had))
+            xs.append(xb.cuda())
+        else:
+            refs.append(oracle.quantize_fp8(x.numpy(), hadamard=had))
+            xs.append(x.cuda())
+        flags.append(had)
+    for _ in range(2):  # the workspace keeps the last call's words: twice in a row
+        codes, ds = zq.quantize_fp8_multi(xs, hadamard=flags)
+        torch.cuda.synchronize()
+        for c, d, (rc, rds) in zip(codes, ds, refs):
+            assert float(d.cpu()[0]) == float(rds)
+            assert np.array_equal(c.view(torch.uint8).cpu().numpy().reshape(rc.shape), rc)
+
+
+def test_quantize_multi_equals_three_single_calls_full_size():
+    # the 32K Gaussian workload's Q, K, V: one multi call against three
+    # per-tensor calls, byte for byte
+    import bf16_causal_prefill_02_b200 as zq
+
+    w = workloads.get("gauss")
+    q, k, v = (t.cuda() for t in workloads.make_inputs(w))
+    codes, ds = zq.quantize_fp8_multi([q, k, v], hadamard=[True, True, False])
+    for x, had, c, d in zip((q, k, v), (True, True, False), codes, ds):
+        c1, d1 = zq.quantize_fp8(x, hadamard=had)
+        torch.cuda.synchronize()
+        assert torch.equal(c.view(torch.uint8), c1.view(torch.uint8))
+        assert torch.equal(d, d1)

@@ -76,12 +76,19 @@ def test_longest_rows_first_inside_head_groups(B, Sq, Sk, Hq, Hkv, causal):
 
 
 @pytest.mark.parametrize("B,S,Hq,Hkv,dqk,dtype,want", [
-    (1, 32768, 32, 32, 128, zq.ZQ_DTYPE_FP8_E4M3, 4),   # K/V 268 MB > 96 MB
-    (1, 4096, 32, 8, 128, zq.ZQ_DTYPE_FP8_E4M3, 32),    # 8 MB: all heads
-    (1, 16384, 16, 16, 192, zq.ZQ_DTYPE_BF16, 4),       # 168 MB
-    (1, 16384, 16, 16, 192, zq.ZQ_DTYPE_FP8_E4M3, 16),  # 84 MB
-    (1, 32768, 6, 6, 128, zq.ZQ_DTYPE_BF16, 6),         # exactly 96 MiB: not above
-    (1, 49152, 6, 6, 128, zq.ZQ_DTYPE_BF16, 2),         # 151 MB, 6 heads: groups of 2
+    # one CTA per unit (more than 64 query tiles): the query heads of one kv head
+    (1, 32768, 32, 32, 128, zq.ZQ_DTYPE_FP8_E4M3, 1),
+    (1, 16384, 32, 8, 128, zq.ZQ_DTYPE_FP8_E4M3, 4),     # 4:1 GQA
+    (1, 16384, 16, 16, 192, zq.ZQ_DTYPE_BF16, 1),
+    (2, 9000, 12, 3, 128, zq.ZQ_DTYPE_BF16, 4),
+    # persistent (at most 64 query tiles): by the size of K/V
+    (1, 4096, 32, 8, 128, zq.ZQ_DTYPE_FP8_E4M3, 32),     # 8 MB: all heads
+    (1, 8192, 32, 32, 128, zq.ZQ_DTYPE_BF16, 4),         # 134 MB > 96 MB
+    (1, 8192, 32, 32, 128, zq.ZQ_DTYPE_FP8_E4M3, 32),    # 67 MB
+    (1, 8192, 6, 6, 128, zq.ZQ_DTYPE_BF16, 6),           # 25 MB
+    (8, 8192, 6, 6, 128, zq.ZQ_DTYPE_BF16, 4),           # 201 MB, 48 heads: groups of 4
+    (4, 8192, 6, 6, 128, zq.ZQ_DTYPE_BF16, 24),          # exactly 96 MiB: not above
+    (1, 8192, 50, 50, 192, zq.ZQ_DTYPE_BF16, 2),         # 262 MB, 50 heads: groups of 2
 ])
 def test_head_group_choice(B, S, Hq, Hkv, dqk, dtype, want):
     plan, _ = zq.attn_plan(B, S, S, Hq, Hkv, d_qk=dqk, dtype=dtype)
