@@ -42,31 +42,35 @@ def test_debug_score_tile_is_qk(dtype, dqk):
     assert err < 1e-5, err
 
 
-def test_debug_leanp_codes_match_emulation():
-    c = Case(1, 128, 128, 1, 1, 128, 128, dtype="leanp", seed=2)
+def _check_p_codes(dtype, seed, std):
+    # every row of the first tile: the GPU's P bytes against the emulation's
+    # p~ encoded back to e4m3 (exact: p~ is an e4m3 value).  The fp32 score
+    # of a key may land on the other side of a rounding boundary than the
+    # fp64 one, so a few codes may differ -- by one code step, never more.
+    c = Case(1, 128, 128, 1, 1, 128, 128, dtype=dtype, seed=seed, std=std)
     _, _, S, P, SF = _debug_run(c)
-    codes = P[:, :32].copy().view(np.uint8).reshape(128, 128)
-    match = total = 0
-    for r in (0, 1, 31, 63, 64, 100, 127):
-        _, _, p = oracle.attn_fp8_emul(c.qd, c.kd, c.vd, mode=oracle.MODE_LEANP, rows=[r], want_p=True)
-        got = oracle.e4m3_decode(codes[r, : r + 1])
-        match += int(np.sum(got == p[: r + 1]))
+    codes = P[:, :32].copy().view(np.uint8).reshape(128, 128).astype(np.int64)
+    mode = oracle.MODE_LEANP if dtype == "leanp" else oracle.MODE_EXACT
+    equal = total = 0
+    for r in range(128):
+        _, _, p = oracle.attn_fp8_emul(c.qd, c.kd, c.vd, mode=mode, rows=[r], want_p=True)
+        ref = oracle.e4m3_encode(p[: r + 1]).astype(np.int64)
+        got = codes[r, : r + 1]
+        assert np.all(np.abs(got - ref) <= 1), (r, np.flatnonzero(np.abs(got - ref) > 1))
+        equal += int(np.sum(got == ref))
         total += r + 1
         assert np.all(codes[r, r + 1 :] == 0)  # masked keys
-    assert match / total >= 0.995, (match, total)
+    assert equal / total >= 0.999, (equal, total)
 
 
-def test_debug_exact_codes_match_emulation():
-    c = Case(1, 128, 128, 1, 1, 128, 128, dtype="exact", seed=3)
-    _, _, S, P, SF = _debug_run(c)
-    codes = P[:, :32].copy().view(np.uint8).reshape(128, 128)
-    match = total = 0
-    for r in (0, 5, 64, 90, 127):
-        _, _, p = oracle.attn_fp8_emul(c.qd, c.kd, c.vd, mode=oracle.MODE_EXACT, rows=[r], want_p=True)
-        got = oracle.e4m3_decode(codes[r, : r + 1])
-        match += int(np.sum(got == p[: r + 1]))
-        total += r + 1
-    assert match / total >= 0.995, (match, total)
+@pytest.mark.parametrize("seed,std", [(2, 1.0), (12, 2.0)])
+def test_debug_leanp_codes_match_emulation(seed, std):
+    _check_p_codes("leanp", seed, std)
+
+
+@pytest.mark.parametrize("seed,std", [(3, 1.0), (13, 2.0)])
+def test_debug_exact_codes_match_emulation(seed, std):
+    _check_p_codes("exact", seed, std)
 
 
 @pytest.mark.parametrize("dtype", DTYPES)

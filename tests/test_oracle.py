@@ -526,3 +526,25 @@ def test_grouped_quantiser_one_slot_is_per_tensor():
     c, d = oracle.quantize_fp8_grouped(x, heads_per_scale=4)
     c1, d1 = oracle.quantize_fp8(x)
     assert np.array_equal(c, c1) and d[0, 0] == d1
+
+
+@pytest.mark.parametrize("mode", [oracle.MODE_EXACT, oracle.MODE_LEANP])
+def test_rotation_reduces_error_with_shared_outlier_channels(mode):
+    # [P2] "Perche l'FP8 non basta da solo": the Hadamard rotation of Q and K
+    # roughly halves the error the input quantisation causes.  On the oracle
+    # alone (R3 quantiser, R2 emulation, R1 on the unquantised inputs): with 4
+    # outlier channels x20 shared by Q and K the error falls below half; with
+    # the rotation the scores are unchanged without quantisation (R1 on the
+    # rotated fp32 inputs, descaled, equals R1 on the originals).
+    w = workloads.get("long_shared", 512)
+    q, k, v = (t.numpy() for t in workloads.make_inputs(w))
+    ref, _ = oracle.attn_ref(q.astype(np.float64), k.astype(np.float64), v.astype(np.float64))
+    err = {}
+    for had in (False, True):
+        deq = []
+        for t, r in ((q, had), (k, had), (v, False)):
+            c, ds = oracle.quantize_fp8(t, hadamard=r)
+            deq.append(oracle.dequant_e4m3(c, float(ds)))
+        o, _ = oracle.attn_fp8_emul(*deq, mode=mode)
+        err[had] = oracle.rel_rmse(o, ref)
+    assert err[True] < 0.5 * err[False], err

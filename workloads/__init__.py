@@ -16,6 +16,11 @@ available, so layer-shaped synthetic tensors stand in for the captured ones):
                                               (theta 1e6); V ~ N(0,1)
   long      B=1 Hq=32 Hkv=8 S=16384 d=128    Q,K = N(0,1), 4 outlier channels
                                               per head x20, then RoPE; V N(0,1)
+  long_shared  as long, but the 4 outlier channels of a kv head are shared
+                                              by its keys and its query heads,
+                                              and Q,K are scaled by
+                                              1/sqrt(1 + 4(20^2 - 1)/d) so that
+                                              E|q|^2 = d as for N(0,1) rows
   mla       B=1 Hq=Hkv=16 S=16384 dqk=192 dv=128   iid N(0,1)
   gauss     B=1 Hq=Hkv=32 d=128, S in {4K,8K,16K,32K}  iid N(0,1)
 """
@@ -35,7 +40,7 @@ class Workload:
     Hkv: int
     dqk: int
     dv: int
-    dist: str  # "iid", "lognormal_rope", "outlier_rope"
+    dist: str  # "iid", "lognormal_rope", "outlier_rope", "shared_outlier_rope"
     seed: int
 
     @property
@@ -60,6 +65,7 @@ WORKLOADS = {
     "long": Workload("long", 1, 16384, 32, 8, 128, 128, "outlier_rope", 2),
     "mla": Workload("mla", 1, 16384, 16, 16, 192, 128, "iid", 3),
     "gauss": Workload("gauss", 1, 32768, 32, 32, 128, 128, "iid", 4),
+    "long_shared": Workload("long_shared", 1, 16384, 32, 8, 128, 128, "shared_outlier_rope", 5),
 }
 
 GAUSS_SWEEP = (4096, 8192, 16384, 32768)
@@ -96,9 +102,28 @@ def _qk(g: torch.Generator, B, S, H, d, dist) -> torch.Tensor:
     return x
 
 
+def _shared_outliers(g: torch.Generator, B, S, Hq, Hkv, d, mult=20.0):
+    """Q and K with 4 outlier channels per kv head, the same channels for the
+    keys of that head and for its query heads, each tensor scaled so that a
+    row's expected squared norm stays d; then RoPE (theta 1e6)."""
+    m = torch.ones((Hkv, d), dtype=torch.float32)
+    for h in range(Hkv):
+        m[h, torch.randperm(d, generator=g)[:4]] = mult
+    norm = 1.0 / float((1.0 + 4.0 * (mult * mult - 1.0) / d) ** 0.5)
+    q = torch.randn((B, S, Hq, d), generator=g, dtype=torch.float32)
+    k = torch.randn((B, S, Hkv, d), generator=g, dtype=torch.float32)
+    q = _rope(q * m.repeat_interleave(Hq // Hkv, dim=0) * norm, 1e6)
+    k = _rope(k * m * norm, 1e6)
+    return q, k
+
+
 def make_inputs(w: Workload, seed: int | None = None):
     """Return fp32 CPU tensors q (B,S,Hq,dqk), k (B,S,Hkv,dqk), v (B,S,Hkv,dv)."""
     g = torch.Generator().manual_seed(w.seed if seed is None else seed)
+    if w.dist == "shared_outlier_rope":
+        q, k = _shared_outliers(g, w.B, w.S, w.Hq, w.Hkv, w.dqk)
+        v = torch.randn((w.B, w.S, w.Hkv, w.dv), generator=g, dtype=torch.float32)
+        return q, k, v
     q = _qk(g, w.B, w.S, w.Hq, w.dqk, w.dist)
     k = _qk(g, w.B, w.S, w.Hkv, w.dqk, w.dist)
     v = torch.randn((w.B, w.S, w.Hkv, w.dv), generator=g, dtype=torch.float32)
