@@ -7,8 +7,9 @@
     python bench.py --gemm-peaks
 
 A step is one pass of the whole hot path over one batch of synthetic input:
-for FP8, the quantisation of Q, K and V (fp32 -> e4m3, three quantiser calls;
-one scale per tensor, or with --descale kv one per (batch, kv head)) followed
+for FP8, the quantisation of Q, K and V (fp32 -> e4m3: one multi-tensor
+quantiser call with one scale per tensor, or with --descale kv three grouped
+calls with one scale per (batch, kv head)) followed
 by the attention kernel; for BF16 the attention kernel alone.  The headline
 workload is the Gaussian peak-sweep point at S = 32768 (B=1, Hq=Hkv=32,
 d=128), FP8 with Lean P and per-64-key block scaling -- the configuration the
@@ -308,12 +309,16 @@ class Step:
             else:
                 self.ds = torch.zeros(3, dtype=torch.float32, device=dev)
                 self.dsq, self.dsk, self.dsv = self.ds[0:1], self.ds[1:2], self.ds[2:3]
-                self.ws = torch.empty(3, zq.zq_quantize_workspace_bytes(), dtype=torch.uint8, device=dev)
+                self.ws = torch.empty(zq.zq_quantize_multi_workspace_bytes(), dtype=torch.uint8, device=dev)
         self.mode = zq.ZQ_SOFTMAX_EXACT if dtype == "exact" else zq.ZQ_SOFTMAX_LEANP
         self.T = T
 
     def launches_per_step(self) -> int:
-        return 1 if self.dtype == "bf16" else 7  # 3 x (amax + write) + attention
+        if self.dtype == "bf16":
+            return 1
+        # per-tensor scales: one amax and one write kernel for Q, K and V
+        # together; per-(batch, kv head) scales: both kernels per tensor
+        return 7 if self.per_kv else 3
 
     def attention(self, out=None):
         zq = self.zq
@@ -335,9 +340,9 @@ class Step:
             zq.quantize_fp8_grouped(self.v32, 1, hadamard=False, out=self.vc, descale=self.dsv,
                                     workspace=self.ws[2])
             return
-        zq.quantize_fp8(self.q32, hadamard=self.hadamard, out=self.qc, descale=self.ds[0:1], workspace=self.ws[0])
-        zq.quantize_fp8(self.k32, hadamard=self.hadamard, out=self.kc, descale=self.ds[1:2], workspace=self.ws[1])
-        zq.quantize_fp8(self.v32, hadamard=False, out=self.vc, descale=self.ds[2:3], workspace=self.ws[2])
+        zq.quantize_fp8_multi([self.q32, self.k32, self.v32], hadamard=[self.hadamard, self.hadamard, False],
+                              outs=[self.qc, self.kc, self.vc], descales=[self.dsq, self.dsk, self.dsv],
+                              workspace=self.ws)
 
     def step(self):
         if self.dtype != "bf16":
