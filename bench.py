@@ -5,6 +5,7 @@
                     [--T T] [--impl reference] [--no-extra] [--no-e2e] [--no-cpu]
                     [--no-energy] [--cpu-seconds SEC]
     python bench.py --gemm-peaks
+    python bench.py --trace [--workload NAME] [--S S] [--dtype ...]
 
 A step is one pass of the whole hot path over one batch of synthetic input:
 for FP8, the quantisation of Q, K and V (fp32 -> e4m3: one multi-tensor
@@ -77,6 +78,8 @@ def parse():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the other workloads measured after the headline (N=1)")
+    ap.add_argument("--trace", action="store_true",
+                    help="only run the debug kernel on one long unit and print its per-role pipeline timing")
     ap.add_argument("--gemm-peaks", action="store_true",
                     help="only measure library FP8 / BF16 GEMM throughput on this GPU and print it")
     return ap.parse_args()
@@ -779,9 +782,72 @@ def gemm_peak_run():
     return res
 
 
+def pipeline_trace(args, w):
+    """Per-role timing of one unit from the debug instantiation's clock64
+    trace (SM cycles), medians over the unit's key tiles 20 .. n-2.  The
+    debug kernel carries the trace stores, so absolute times run a little
+    long; the shares between roles are the point.  Slots: softmax warp 0
+    saw S_j [0], loaded it [1], computed P_j [2], released it [3]; warps 3,
+    1, 5 released P_j [4], [11], [12] (warps 1 and 5 share their SM
+    sub-partition with the MMA issuer); MMA issuer: K_j landed and QK_j
+    issue starts [5], QK_j issued and committed [6], P_j seen [7], scales
+    copied [8], PV_j issued [9] and committed [10]."""
+    import bf16_causal_prefill_02_b200 as zq
+
+    step = Step(w, args.dtype, args.hadamard, T=args.T)
+    step.step()
+    torch.cuda.synchronize()
+    n_tiles = (w.S + 127) // 128
+    t = min(n_tiles - 1, 200)
+    bh = min(5, w.B * w.Hq - 1)
+    dbg = torch.zeros(zq.ZQ_DEBUG_BYTES // 4, dtype=torch.int32, device="cuda")
+    kw = dict(out=step.out, lse=step.lse, debug=dbg, debug_at=(bh, t))
+    if args.dtype == "bf16":
+        zq.attn_fwd(step.qb, step.kb, step.vb, **kw)
+    else:
+        zq.attn_fwd(step.qc, step.kc, step.vc, q_descale=step.dsq, k_descale=step.dsk, v_descale=step.dsv,
+                    softmax_mode=step.mode, block_scale=True, headroom_T=step.T, **kw)
+    torch.cuda.synchronize()
+    off = 128 * 128 + 128 * 64 + 256
+    tr = dbg[off:].cpu().numpy().view(np.uint64)[: 512 * 16].reshape(512, 16).astype(np.int64)
+    n = t + 1 if w.S > 0 else 0
+    lo, hi = 20, n - 2
+    if hi - lo < 8:
+        lo, hi = 1, n - 2
+    r = tr[lo:hi]
+    nxt = tr[lo + 2:hi + 2]
+    med = lambda x: float(np.median(x))
+    rel = np.stack([r[:, 3], r[:, 4], r[:, 11], r[:, 12]], axis=1)
+    last = rel.max(axis=1)
+    out = {
+        "trace": "%s tile %d of flat head %d (%d key tiles), SM cycles, medians over tiles %d..%d"
+                 % (w.name + "_" + args.dtype, t, bh, n, lo, hi - 1),
+        "period_cycles": med(np.diff(tr[lo:hi + 1, 3])),
+        "softmax": {"S_ready_after_QK_commit_issue": med(r[:, 0] - r[:, 6]),
+                    "S_load": med(r[:, 1] - r[:, 0]), "P_compute": med(r[:, 2] - r[:, 1]),
+                    "P_store_and_release_warp0": med(r[:, 3] - r[:, 2]),
+                    "release_after_warp0": {"warp3": med(r[:, 4] - r[:, 3]), "warp1": med(r[:, 11] - r[:, 3]),
+                                            "warp5": med(r[:, 12] - r[:, 3])}},
+        "mma": {"P_seen_after_last_release": med(r[:, 7] - last), "scales_copied": med(r[:, 8] - r[:, 7]),
+                "PV_issued": med(r[:, 9] - r[:, 8]), "PV_committed": med(r[:, 10] - r[:, 9]),
+                "next_QK_start_after_PV_commit": med(nxt[:, 5] - r[:, 10]),
+                "QK_issue": med(r[:, 6] - r[:, 5])},
+    }
+    out["share_of_period"] = {
+        "softmax_warp0_busy": round((out["softmax"]["S_load"] + out["softmax"]["P_compute"] +
+                                     out["softmax"]["P_store_and_release_warp0"]) / out["period_cycles"], 3),
+        "last_release_lag": round(med(last - r[:, 3]) / out["period_cycles"], 3),
+        "mma_issue_PV_and_QK": round((med(r[:, 9] - r[:, 7]) + out["mma"]["QK_issue"]) / out["period_cycles"], 3)}
+    return out
+
+
 def main():
     args = parse()
     w = workloads.get(args.workload, args.S)
+    if args.trace:
+        torch.cuda.set_device(0)
+        print(json.dumps(pipeline_trace(args, w)), flush=True)
+        return
     if args.gemm_peaks:
         torch.cuda.set_device(0)
         print(json.dumps(gemm_peak_run()), flush=True)
