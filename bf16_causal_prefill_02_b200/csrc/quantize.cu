@@ -459,10 +459,17 @@ __device__ __forceinline__ float amax192_part(const void* x, int64_t n_vec, int6
   return m;
 }
 
+// The write pass walks each thread's elements in the reverse order of the
+// amax pass: the grid covers the tensor in rounds of nthreads * 4 elements,
+// and the rounds the amax pass read last are the likeliest to still sit in
+// L2 (the three tensors of a 4K call fit in it).
 template <bool BF16IN, bool HAD>
 __device__ __forceinline__ void write_part(const void* x, int64_t n, float inv, uint8_t* out, int64_t t0,
                                            int64_t nthreads, int lane) {
-  for (int64_t i = t0 * 4; i < n; i += nthreads * 4) {
+  const int64_t step = nthreads * 4;
+  if (t0 * 4 >= n) return;
+  for (int64_t r = (n - t0 * 4 + step - 1) / step - 1; r >= 0; --r) {
+    const int64_t i = t0 * 4 + r * step;
     float v[4];
     load4<BF16IN>(x, i, v);
     if constexpr (HAD) fwht128_warp(v, lane);
@@ -473,7 +480,9 @@ __device__ __forceinline__ void write_part(const void* x, int64_t n, float inv, 
 template <bool BF16IN>
 __device__ __forceinline__ void write192_part(const void* x, int64_t n_vec, float inv, uint8_t* out, int64_t w0,
                                               int64_t nwarps, int lane) {
-  for (int64_t vec = w0; vec < n_vec; vec += nwarps) {
+  if (w0 >= n_vec) return;
+  for (int64_t r = (n_vec - w0 + nwarps - 1) / nwarps - 1; r >= 0; --r) {  // reverse rounds, as write_part
+    const int64_t vec = w0 + r * nwarps;
     float a[4], c[2];
     load4<BF16IN>(x, vec * 192 + 4 * lane, a);
     load2<BF16IN>(x, vec * 192 + 128 + 2 * lane, c);
