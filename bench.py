@@ -233,14 +233,14 @@ def cpu_model() -> str:
 
 
 def kernel_sources_digest(read=None) -> str:
-    """sha256 over the attention kernel's sources: attn_fwd.cu and every
-    header beside it, by name in sorted order.  `read(name)` returns a
-    file's bytes (default: the files in csrc)."""
+    """sha256 over the attention kernels' sources: attn_fwd.cu, attn_pp.cu
+    and every header beside them, by name in sorted order.  `read(name)`
+    returns a file's bytes (default: the files in csrc)."""
     import hashlib
 
     csrc = os.path.join(ROOT, "bf16_causal_prefill_02_b200", "csrc")
     if read is None:
-        names = sorted(n for n in os.listdir(csrc) if n == "attn_fwd.cu" or n.endswith((".h", ".cuh")))
+        names = sorted(n for n in os.listdir(csrc) if n in ("attn_fwd.cu", "attn_pp.cu") or n.endswith((".h", ".cuh")))
 
         def read(n):
             with open(os.path.join(csrc, n), "rb") as f:
@@ -619,11 +619,17 @@ def config_dict(w, args, world):
             "parallelism": "dp%d (independent batches, no collective)" % world}
 
 
-def roofline_dict(kind, flops, m, tkey):
+def attention_kernel_name(kind, dqk):
+    """The kernel launch_attention runs: the paired one (two query tiles per
+    CTA) for BF16 at d = 128, else the single-tile one."""
+    return "attn_pp_kernel" if kind == "bf16" and dqk == 128 else "attn_fwd_kernel"
+
+
+def roofline_dict(kind, flops, m, tkey, dqk=128):
     peak, peak_src = tensor_peak(kind)
     achieved = flops / (m["attn_ms"] * 1e-3) / 1e12
     traffic, traffic_stale = load_traffic(tkey)
-    r = {"bound": "tensor", "kernel": "attn_fwd_kernel", "achieved": round(achieved, 1),
+    r = {"bound": "tensor", "kernel": attention_kernel_name(kind, dqk), "achieved": round(achieved, 1),
          "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
          "peak_source": peak_src,
          "frac_of_datasheet_dense": round(achieved / DATASHEET_DENSE_TFLOPS[kind], 4),
@@ -676,7 +682,7 @@ def run_ours(args, rank, world, w):
         "scaling": "weak", "vs_baseline": None,
         "dtype": "fp8_e4m3" if kind == "fp8" else "bf16", "data": "synthetic",
         "config": config_dict(w, args, world),
-        "roofline": roofline_dict(kind, flops, m, tkey),
+        "roofline": roofline_dict(kind, flops, m, tkey, w.dqk),
         "clocks": m["clocks"],
         "energy": m["energy"],
         "e2e": e2e,
@@ -782,6 +788,31 @@ def gemm_peak_run():
     return res
 
 
+def _pair_trace(dbg, off, w, args, t, bh):
+    """The paired kernel's trace (one team: the traced 128-row tile t):
+    per 64-key tile j, team slots [0] S_j seen, [1] loaded, [2] P_j
+    computed, [3] released (warp 0 of the team); its issuer: [4] QK_j issue
+    starts, [5] QK_j committed, [6] P_j seen, [7] PV_j committed."""
+    tr = dbg[off:].cpu().numpy().view(np.uint64)[: 512 * 16].reshape(512, 2, 8)[:, t & 1].astype(np.int64)
+    n = min((128 * t + 127) // 64 + 1, 512)
+    lo, hi = 20, n - 2
+    if hi - lo < 8:
+        lo, hi = 1, n - 2
+    r, nxt = tr[lo:hi], tr[lo + 1:hi + 1]
+    med = lambda x: float(np.median(x))
+    out = {
+        "trace": "%s tile %d of flat head %d (team %d of its pair, %d key tiles of 64), SM cycles, medians over "
+                 "tiles %d..%d" % (w.name + "_" + args.dtype, t, bh, t & 1, n, lo, hi - 1),
+        "period_cycles": med(np.diff(tr[lo:hi + 1, 3])),
+        "softmax": {"S_ready_after_QK_commit_issue": med(r[:, 0] - r[:, 5]), "S_load": med(r[:, 1] - r[:, 0]),
+                    "P_compute": med(r[:, 2] - r[:, 1]), "P_store_and_release": med(r[:, 3] - r[:, 2]),
+                    "next_S_seen_after_release": med(nxt[:, 0] - r[:, 3])},
+        "issuer": {"P_seen_after_release": med(r[:, 6] - r[:, 3]), "PV_issue": med(r[:, 7] - r[:, 6]),
+                   "next_QK_start_after_S_load": med(nxt[:, 4] - r[:, 1]), "QK_issue": med(r[:, 5] - r[:, 4])},
+    }
+    return out
+
+
 def pipeline_trace(args, w):
     """Per-role timing of one unit from the debug instantiation's clock64
     trace (SM cycles), medians over the unit's key tiles 20 .. n-2.  The
@@ -809,6 +840,8 @@ def pipeline_trace(args, w):
                     softmax_mode=step.mode, block_scale=True, headroom_T=step.T, **kw)
     torch.cuda.synchronize()
     off = 128 * 128 + 128 * 64 + 256
+    if attention_kernel_name("bf16" if args.dtype == "bf16" else "fp8", w.dqk) == "attn_pp_kernel":
+        return _pair_trace(dbg, off, w, args, t, bh)
     tr = dbg[off:].cpu().numpy().view(np.uint64)[: 512 * 16].reshape(512, 16).astype(np.int64)
     n = t + 1 if w.S > 0 else 0
     lo, hi = 20, n - 2

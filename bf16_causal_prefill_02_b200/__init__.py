@@ -62,6 +62,7 @@ class zq_attn_plan(ctypes.Structure):
     _fields_ = [
         ("n_units", ctypes.c_int64), ("grid", ctypes.c_int64), ("persistent", ctypes.c_int),
         ("head_group", ctypes.c_int), ("smem_bytes", ctypes.c_int), ("threads", ctypes.c_int),
+        ("rows_per_unit", ctypes.c_int), ("keys_per_tile", ctypes.c_int),
     ]
 
 

@@ -20,8 +20,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 OUT = os.path.join(HERE, "libzattn.so")
 BUILD_DIR = os.path.join(ROOT, "_build")
-SOURCES = ["zattn_api.cu", "quantize.cu", "attn_fwd.cu"]
-HEADERS = ["sm100_ptx.cuh", "zq_internal.h", "schedule.h"]
+SOURCES = ["zattn_api.cu", "quantize.cu", "attn_fwd.cu", "attn_pp.cu"]
+HEADERS = ["sm100_ptx.cuh", "zq_internal.h", "schedule.h", "attn_math.cuh"]
 
 
 def nvcc() -> str:

@@ -44,6 +44,49 @@ __host__ __device__ __forceinline__ Unit unit_of(const AttnParams& p, int u) {
   return w;
 }
 
+// The paired kernel's unit: two consecutive 128-row query tiles 2tp and
+// 2tp + 1 of one flat head, one per softmax team, sharing every K/V tile.
+// Keys come in tiles of 64 (kPairKeyTile).  Numbering as for Unit (groups
+// of head_group flat heads, longest rows first), over (n_qtiles + 1) / 2
+// pairs per head.  Team t visits key tiles 0 .. n_kv[t] - 1; the second
+// tile's rows are later, so n_kv[1] >= n_kv[0] whenever the second tile
+// has rows (a tile past Sq has none: n_kv = 0).
+constexpr int kPairKeyTile = 64;
+struct PairUnit {
+  int tp, bh, b, h, g;
+  int q0[2], n_kv[2], min_lim[2];
+  int n_kv_max;
+};
+__host__ __device__ __forceinline__ int n_pairs_of(int n_qtiles) { return (n_qtiles + 1) / 2; }
+__host__ __device__ __forceinline__ PairUnit pair_of(const AttnParams& p, int u) {
+  PairUnit w;
+  const int GH = p.head_group;
+  const int np = n_pairs_of(p.n_qtiles);
+  const int gi = u / (GH * np), gr = u % (GH * np);
+  w.tp = np - 1 - gr / GH;
+  w.bh = gi * GH + gr % GH;
+  w.b = w.bh / p.Hq;
+  w.h = w.bh % p.Hq;
+  w.g = w.h / (p.Hq / p.Hkv);
+  const int shift = p.Sk - p.Sq;
+  w.n_kv_max = 0;
+  for (int t = 0; t < 2; ++t) {
+    const int q0 = (2 * w.tp + t) * kTile;
+    w.q0[t] = q0;
+    if (q0 >= p.Sq) {
+      w.n_kv[t] = 0;
+      w.min_lim[t] = -1;
+      continue;
+    }
+    const int q1 = min(q0 + kTile - 1, p.Sq - 1);
+    const int max_key = p.causal ? min(q1 + shift, p.Sk - 1) : p.Sk - 1;
+    w.n_kv[t] = max_key < 0 ? 0 : max_key / kPairKeyTile + 1;
+    w.min_lim[t] = p.causal ? min(q0 + shift, p.Sk - 1) : p.Sk - 1;
+    w.n_kv_max = max(w.n_kv_max, w.n_kv[t]);
+  }
+  return w;
+}
+
 // The k-th unit of CTA `cta` among `grid` persistent CTAs: rounds of `grid`
 // units, walked forwards in even rounds and backwards in odd ones, so that
 // under longest-rows-first numbering every CTA pairs long units with short

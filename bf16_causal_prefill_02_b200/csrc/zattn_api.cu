@@ -158,20 +158,33 @@ int zq_attn_plan_launch(const zq_attn_args* a, int num_sms, zq_attn_plan* plan,
   }
   const zq::AttnLaunch L = make_launch(a);
   const zq::AttnParams& p = L.p;
-  const long long n_units = (long long)p.n_qtiles * p.B * p.Hq;
+  // the kernel launch_attention picks: pairs of query tiles with 64-key
+  // tiles (BF16, d = 128, more than 64 query tiles), else single query
+  // tiles with 128-key tiles
+  const bool pair = zq::use_pair_kernel(L.dtype, L.dqk, p.n_qtiles);
+  const long long n_units = (long long)(pair ? zq::n_pairs_of(p.n_qtiles) : p.n_qtiles) * p.B * p.Hq;
   const long long grid = zq::grid_size(p.n_qtiles, n_units, num_sms);
   plan->n_units = n_units;
   plan->grid = grid;
   plan->persistent = zq::use_persistent(p.n_qtiles) ? 1 : 0;
   plan->head_group = p.head_group;
-  plan->smem_bytes = zq::attn_smem_bytes(a->dtype, a->d_qk);
-  plan->threads = zq::attn_threads();
+  plan->smem_bytes = pair ? zq::attn_pp_smem_bytes() : zq::attn_smem_bytes(a->dtype, a->d_qk);
+  plan->threads = pair ? zq::attn_pp_threads() : zq::attn_threads();
+  plan->rows_per_unit = pair ? 2 * zq::kTile : zq::kTile;
+  plan->keys_per_tile = pair ? zq::kPairKeyTile : zq::kTile;
   if (!unit_tile && !unit_bh && !unit_nkv && !unit_cta && !unit_round) return ZQ_OK;
   for (long long u = 0; u < n_units; ++u) {
-    const zq::Unit w = zq::unit_of(p, (int)u);
-    if (unit_tile) unit_tile[u] = w.t;
-    if (unit_bh) unit_bh[u] = w.bh;
-    if (unit_nkv) unit_nkv[u] = w.n_kv;
+    int t, bh, nkv;
+    if (pair) {
+      const zq::PairUnit w = zq::pair_of(p, (int)u);
+      t = w.tp, bh = w.bh, nkv = w.n_kv_max;
+    } else {
+      const zq::Unit w = zq::unit_of(p, (int)u);
+      t = w.t, bh = w.bh, nkv = w.n_kv;
+    }
+    if (unit_tile) unit_tile[u] = t;
+    if (unit_bh) unit_bh[u] = bh;
+    if (unit_nkv) unit_nkv[u] = nkv;
   }
   if (unit_cta || unit_round) {
     // walk every CTA's sequence exactly as the kernel does

@@ -51,6 +51,13 @@ struct AttnLaunch {
 };
 
 cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t st);
+// the paired kernel (two 128-row query tiles per CTA, 64-key tiles, one
+// CTA per unit): BF16 at d_qk = d_v = 128 with more than 64 query tiles;
+// launch_attention dispatches to it
+bool use_pair_kernel(int dtype, int dqk, int n_qtiles);
+cudaError_t launch_attention_pp(const AttnLaunch& a, cudaStream_t st);
+int attn_pp_smem_bytes();
+int attn_pp_threads();
 // dynamic shared memory and threads of one attention CTA (host side)
 int attn_smem_bytes(int dtype, int dqk);
 int attn_threads();

@@ -148,12 +148,15 @@ ZQ_API int zq_attn_fwd_ex(const zq_attn_args* args, void* stream);
 
 /* Launch shape of one attention call, from zq_attn_plan_launch. */
 typedef struct zq_attn_plan {
-  int64_t n_units;  /* work units: ceil(Sq / 128) query tiles x B x Hq        */
-  int64_t grid;     /* CTAs launched                                          */
-  int persistent;   /* 1: each CTA walks several units (Sq <= 64 x 128 rows)  */
-  int head_group;   /* flat heads whose tiles are interleaved in unit order  */
-  int smem_bytes;   /* dynamic shared memory per CTA                          */
-  int threads;      /* threads per CTA                                        */
+  int64_t n_units;   /* work units: ceil(Sq / rows_per_unit) x B x Hq          */
+  int64_t grid;      /* CTAs launched                                          */
+  int persistent;    /* 1: each CTA walks several units (Sq <= 64 x 128 rows)  */
+  int head_group;    /* flat heads whose tiles are interleaved in unit order  */
+  int smem_bytes;    /* dynamic shared memory per CTA                          */
+  int threads;       /* threads per CTA                                        */
+  int rows_per_unit; /* query rows per unit: 128, or 256 (BF16 at d_qk = d_v =
+                        128: a pair of 128-row tiles, one per softmax team)    */
+  int keys_per_tile; /* keys per key tile: 128, or 64 with 256-row units       */
 } zq_attn_plan;
 
 /*
@@ -172,10 +175,13 @@ typedef struct zq_attn_plan {
  *   unit_tile, unit_bh, unit_nkv, unit_cta, unit_round: optional HOST
  *             arrays of plan->n_units int32 each (NULL to skip; call once
  *             with all NULL to learn n_units).  Entry u describes work unit
- *             u: its query tile t (rows 128t..128t+127), its flat head
- *             b * Hq + h, the number of key tiles it visits (tiles
- *             0..n_kv-1), the CTA that runs it and its position in that
- *             CTA's sequence.  Units are numbered in groups of head_group
+ *             u: its index t along the query axis (rows
+ *             rows_per_unit * t ..  + rows_per_unit - 1), its flat head
+ *             b * Hq + h, the number of key tiles of keys_per_tile keys it
+ *             visits (tiles 0..n_kv-1; with 256-row units the later 128-row
+ *             tile's count, the earlier one stopping at its own diagonal),
+ *             the CTA that runs it and its position in that CTA's
+ *             sequence.  Units are numbered in groups of head_group
  *             heads, longest rows first inside a group; a persistent CTA c
  *             of G runs, in round k, unit k*G + c (k even) or
  *             k*G + G-1-c (k odd).
@@ -195,8 +201,11 @@ ZQ_API int zq_attn_plan_launch(const zq_attn_args* args, int num_sms, zq_attn_pl
  * words hold 4 x e4m3 each, key order little-endian), uint32 SF[2][128]
  * (FP8: the UE8M0 scale of 64-key block 0 / 1 of each row, repeated in all
  * four bytes), then uint64 TRACE[512][16]: SM clock (clock64) at up to sixteen points of
- * the pipeline for key tile j (see attn_fwd.cu).  flags: 0, or 1 to make
- * the MMA issuer withhold all work so that every other role's bounded wait
+ * the pipeline for key tile j (see attn_fwd.cu); with 256-row units
+ * (zq_attn_plan.rows_per_unit, BF16 at d = 128) TRACE[512][2][8] for 64-key
+ * tile j, the traced tile's team t = dbg_qtile & 1 in [j][t] (see
+ * attn_pp.cu).  flags: 0, or 1 to make
+ * the MMA issuers withhold all work so that every other role's bounded wait
  * runs out: the kernel then writes ZQ_ERR_TIMEOUT to args->status and
  * returns (about two seconds later) with the outputs undefined; nothing
  * faults or hangs.  For tests and tuning. */

@@ -138,3 +138,72 @@ def test_plan_argument_errors():
     assert zq._lib.zq_attn_plan_launch(a, 148, None, None, None, None, None, None) == zq.ZQ_ERR_NULL
     a.d_qk = 64
     assert zq.zq_attn_plan_launch(a, 148, zq.zq_attn_plan()) == zq.ZQ_ERR_UNSUPPORTED
+
+
+# ------------------------------------------------- paired units (BF16, d = 128)
+LONG = [
+    # B, Sq, Sk, Hq, Hkv, causal: more than 64 query tiles (one CTA per unit)
+    (1, 8320, 8320, 2, 1, True),      # 65 tiles: the last pair has one tile
+    (1, 9000, 12000, 3, 3, True),     # Sq < Sk
+    (1, 12000, 9000, 2, 2, True),     # Sq > Sk: the first rows see no key
+    (2, 8500, 8700, 2, 1, False),
+    (1, 32768, 32768, 32, 32, True),
+]
+
+
+def _brute_n_kv_rows(r0, r1, Sq, Sk, causal, kt):
+    """Key tiles of kt keys holding a key visible to some query row in [r0, r1)."""
+    rows = np.arange(r0, min(r1, Sq))
+    if rows.size == 0:
+        return 0
+    if not causal:
+        return (Sk + kt - 1) // kt
+    last = min(int(rows.max()) + Sk - Sq, Sk - 1)  # visible keys of the last row form a prefix
+    return 0 if last < 0 else last // kt + 1
+
+
+@pytest.mark.parametrize("B,Sq,Sk,Hq,Hkv,causal", LONG)
+def test_long_bf16_d128_units_are_tile_pairs(B, Sq, Sk, Hq, Hkv, causal):
+    # BF16 at d = 128 with more than 64 query tiles runs the paired kernel:
+    # a unit is two consecutive 128-row tiles (256 rows) with 64-key tiles,
+    # one CTA per unit; every pair once, longest rows first in head groups
+    plan, u = zq.attn_plan(B, Sq, Sk, Hq, Hkv, dtype=zq.ZQ_DTYPE_BF16, causal=causal, num_sms=148)
+    npairs = ((Sq + 127) // 128 + 1) // 2
+    assert plan.rows_per_unit == 256 and plan.keys_per_tile == 64
+    assert plan.n_units == npairs * B * Hq and plan.persistent == 0 and plan.grid == plan.n_units
+    assert plan.threads == 352 and 0 < plan.smem_bytes <= 227 * 1024
+    assert set(zip(u["tile"].tolist(), u["bh"].tolist())) == {(t, bh) for t in range(npairs) for bh in range(B * Hq)}
+    GH = plan.head_group
+    for gi in range(B * Hq // GH):
+        sl = slice(gi * GH * npairs, (gi + 1) * GH * npairs)
+        assert np.array_equal(u["tile"][sl], np.repeat(np.arange(npairs - 1, -1, -1), GH))
+    assert np.array_equal(u["cta"], np.arange(plan.n_units)) and not u["round"].any()
+
+
+@pytest.mark.parametrize("B,Sq,Sk,Hq,Hkv,causal", LONG[:4])
+def test_pair_causal_skip_matches_brute_force(B, Sq, Sk, Hq, Hkv, causal):
+    # a pair visits the 64-key tiles its later tile needs; the earlier tile
+    # stops at its own diagonal (the kernel's parity tests check the rows)
+    _, u = zq.attn_plan(B, Sq, Sk, Hq, Hkv, dtype=zq.ZQ_DTYPE_BF16, causal=causal)
+    for t, n in zip(u["tile"].tolist(), u["n_kv"].tolist()):
+        assert n == _brute_n_kv_rows(256 * t, 256 * t + 256, Sq, Sk, causal, 64), (t, n)
+
+
+def test_pair_counts_at_32k():
+    # S = 32768: pair t visits 4t + 4 key tiles of 64 keys
+    _, u = zq.attn_plan(1, 32768, 32768, 32, 32, dtype=zq.ZQ_DTYPE_BF16)
+    assert np.array_equal(u["n_kv"], 4 * u["tile"] + 4)
+    assert int(u["n_kv"].sum()) == 32 * 4 * 128 * 129 // 2
+
+
+@pytest.mark.parametrize("B,S,dtype,dqk", [
+    (1, 8192, zq.ZQ_DTYPE_BF16, 128),       # 64 tiles: persistent, single-tile kernel
+    (2, 1000, zq.ZQ_DTYPE_BF16, 128),
+    (1, 16384, zq.ZQ_DTYPE_BF16, 192),      # MLA
+    (1, 16384, zq.ZQ_DTYPE_FP8_E4M3, 128),  # FP8
+    (1, 16384, zq.ZQ_DTYPE_FP8_E4M3, 192),
+])
+def test_other_shapes_keep_single_tile_units(B, S, dtype, dqk):
+    plan, u = zq.attn_plan(B, S, S, 4, 2, d_qk=dqk, dtype=dtype)
+    assert plan.rows_per_unit == 128 and plan.keys_per_tile == 128 and plan.threads == 320
+    assert plan.n_units == (S + 127) // 128 * B * 4
