@@ -619,17 +619,18 @@ def config_dict(w, args, world):
             "parallelism": "dp%d (independent batches, no collective)" % world}
 
 
-def attention_kernel_name(kind, dqk):
+def attention_kernel_name(kind, dqk, sq):
     """The kernel launch_attention runs: the paired one (two query tiles per
-    CTA) for BF16 at d = 128, else the single-tile one."""
-    return "attn_pp_kernel" if kind == "bf16" and dqk == 128 else "attn_fwd_kernel"
+    CTA) for BF16 at d = 128 with more than 64 query tiles of 128 rows, else
+    the single-tile one."""
+    return "attn_pp_kernel" if kind == "bf16" and dqk == 128 and (sq + 127) // 128 > 64 else "attn_fwd_kernel"
 
 
-def roofline_dict(kind, flops, m, tkey, dqk=128):
+def roofline_dict(kind, flops, m, tkey, dqk, sq):
     peak, peak_src = tensor_peak(kind)
     achieved = flops / (m["attn_ms"] * 1e-3) / 1e12
     traffic, traffic_stale = load_traffic(tkey)
-    r = {"bound": "tensor", "kernel": attention_kernel_name(kind, dqk), "achieved": round(achieved, 1),
+    r = {"bound": "tensor", "kernel": attention_kernel_name(kind, dqk, sq), "achieved": round(achieved, 1),
          "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
          "peak_source": peak_src,
          "frac_of_datasheet_dense": round(achieved / DATASHEET_DENSE_TFLOPS[kind], 4),
@@ -682,7 +683,7 @@ def run_ours(args, rank, world, w):
         "scaling": "weak", "vs_baseline": None,
         "dtype": "fp8_e4m3" if kind == "fp8" else "bf16", "data": "synthetic",
         "config": config_dict(w, args, world),
-        "roofline": roofline_dict(kind, flops, m, tkey, w.dqk),
+        "roofline": roofline_dict(kind, flops, m, tkey, w.dqk, w.S),
         "clocks": m["clocks"],
         "energy": m["energy"],
         "e2e": e2e,
@@ -840,7 +841,7 @@ def pipeline_trace(args, w):
                     softmax_mode=step.mode, block_scale=True, headroom_T=step.T, **kw)
     torch.cuda.synchronize()
     off = 128 * 128 + 128 * 64 + 256
-    if attention_kernel_name("bf16" if args.dtype == "bf16" else "fp8", w.dqk) == "attn_pp_kernel":
+    if attention_kernel_name("bf16" if args.dtype == "bf16" else "fp8", w.dqk, w.S) == "attn_pp_kernel":
         return _pair_trace(dbg, off, w, args, t, bh)
     tr = dbg[off:].cpu().numpy().view(np.uint64)[: 512 * 16].reshape(512, 16).astype(np.int64)
     n = t + 1 if w.S > 0 else 0

@@ -90,3 +90,18 @@ def test_reference_arm_config_matches_ours():
     for key in ("block_scale", "headroom_T", "step", "l2", "parallelism"):
         assert key in ours
     assert lines[0]["cpu_baseline"]["cpu_model"]
+
+
+def test_attention_kernel_name_follows_the_library_dispatch():
+    # the bench names the kernel the library runs: the paired kernel for
+    # BF16 at d = 128 beyond 64 query tiles, the single-tile one otherwise
+    # (zq_attn_plan_launch reports the same choice as rows_per_unit)
+    import bench
+    import bf16_causal_prefill_02_b200 as zq
+
+    for kind, dqk, S in (("bf16", 128, 32768), ("bf16", 128, 8192), ("bf16", 128, 8193), ("bf16", 192, 16384),
+                         ("fp8", 128, 32768), ("fp8", 192, 16384)):
+        plan, _ = zq.attn_plan(1, S, S, 2, 2, d_qk=dqk,
+                               dtype=zq.ZQ_DTYPE_BF16 if kind == "bf16" else zq.ZQ_DTYPE_FP8_E4M3)
+        want = "attn_pp_kernel" if plan.rows_per_unit == 256 else "attn_fwd_kernel"
+        assert bench.attention_kernel_name(kind, dqk, S) == want, (kind, dqk, S)
