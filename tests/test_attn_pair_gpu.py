@@ -42,6 +42,9 @@ def _uses_pair_kernel(case):
     (1, 12000, 9000, 2, 2, True),     # Sq > Sk: the first 3000 rows see no key
     (2, 8500, 8700, 2, 1, False),     # non-causal, GQA, a ragged last key tile
     (1, 8448, 8448, 4, 1, True),      # 4:1 GQA, 66 tiles
+    (1, 8193, 8193, 1, 1, True),      # the last tile holds one row
+    (1, 9000, 1, 2, 2, True),         # one key: only the last row sees it
+    (1, 9000, 70, 1, 1, False),       # fewer keys than one key tile, non-causal
 ])
 def test_pair_kernel_sampled_rows(B, Sq, Sk, Hq, Hkv, causal):
     c = Case(B, Sq, Sk, Hq, Hkv, 128, 128, dtype="bf16", causal=causal, seed=Sq % 97 + Sk % 89)
