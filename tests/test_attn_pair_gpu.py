@@ -20,7 +20,7 @@ def _rows(B, Hq, Sq, every=97):
     and of the first pair (both teams, the diagonal tiles, the ragged end)."""
     nq = (Sq + 127) // 128
     tiles = sorted(set(range(max(0, nq - 8), nq)) | {0, 1})
-    edge = sorted({i for t in tiles for i in (128 * t, 128 * t + 1, min(128 * t + 127, Sq - 1))})
+    edge = sorted({i for t in tiles for i in (128 * t, 128 * t + 1, 128 * t + 127) if i < Sq})
     rows = []
     for bh in range(B * Hq):
         idx = sorted(set(range(bh % 7, Sq, every)) | set(edge) | {Sq - 1})
